@@ -1,0 +1,348 @@
+/*
+ * lf_oracle.c -- plain, slow, single-threaded fp64 reference of the Light Forcing
+ * Hierarchical Sparse Attention (HSA) call and of the Chunk-Aware Growth (CAG)
+ * budget solver.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path may call this file: only
+ * the tests, the package's smoke check and the benchmark's CPU-baseline leg load
+ * it. It shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (the pages are summaries of arXiv 2602.04789):
+ *   [RB]  "Light Forcing：通过稀疏注意力加速自回归视频扩散" (paper.rainbus.top),
+ *         execution-flow paragraph: stage 1 (CAG sparsity s_i = s_base - alpha_i*beta,
+ *         first chunk dense, beta fixed by the total-FLOPs constraint), stage 2
+ *         (block mean pooling of q and k, frame pooling of memory keys), stage 3
+ *         (frame scores p_r = <q~_r, k^_M>, top-k frames T_r with the sink, most
+ *         recent and current-chunk frames always kept, block scores
+ *         o_r(tau,j) = <q~_r, k~_j^(tau)>, top-k blocks J_r(tau), mask
+ *         B_r(tau,j) = 1[tau in T_r, j in J_r(tau)], block-sparse attention).
+ *   [GS]  "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
+ *         Attention" (gist.science), Technical Summary sections 2.1 (CAG) and 2.2
+ *         (HSA: mean pooling at block and frame granularity, two-level selection,
+ *         fixed attention cost per query block).
+ *   [NE]  "南洋理工大学打造视频生成新引擎" (163.com), section 2 (CAG: weighted
+ *         sparsities meet the target budget) and section 3 (HSA stages).
+ *
+ * Readings where the pages are silent (each is listed with its reason in the
+ * design notes): blocks never straddle frames and the last block of a frame may
+ * be partial; frame pooling is the token mean of the whole frame; ties in every
+ * top-k go to the lower index; block top-k applies inside every selected frame,
+ * forced ones included; selection is per (batch, head, query block); scores are
+ * plain inner products; attention uses scale/softmax over exactly the valid
+ * tokens of the kept blocks with no causal mask; a query block with an empty
+ * list gets a zero output.
+ *
+ * Inputs q, k, v are bf16 bit patterns (uint16). Step 1 of every routine converts
+ * them to fp64 exactly; all arithmetic after that is fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- exact bf16 -> fp64 ------------------------------------------------- */
+static double bf16_to_f64(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+/* Tokens [t0, t1) of block j of a frame (frame-relative). */
+static void block_span(int F, int bt, int j, int* t0, int* t1)
+{
+    *t0 = j * bt;
+    *t1 = (j + 1) * bt < F ? (j + 1) * bt : F;
+}
+
+/* ---- stage 2: token compression (mean pooling) --------------------------- */
+/*
+ * [RB] stage 2; [GS] 2.2 "Token Compression".
+ * q_pool[b,h,r,:]  = mean of the query tokens of query block r
+ * k_pool[b,h,g,:]  = mean of the key tokens of KV block g = tau*bpf + j
+ * k_frame[b,h,tau,:] = mean of all key tokens of frame tau
+ * k and v rows of head (b,h) start at (b*H + h) * kv_stride tokens.
+ */
+void orc_pool(int B, int H, int D, int F, int bt, int NF, int n_cur, long kv_stride,
+              const uint16_t* q, const uint16_t* k,
+              double* q_pool, double* k_pool, double* k_frame)
+{
+    int bpf = ceil_div(F, bt);
+    long Lq = (long)n_cur * F;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            long bh = (long)b * H + h;
+            const uint16_t* qh = q + bh * Lq * D;
+            const uint16_t* kh = k + bh * kv_stride * D;
+            /* query blocks */
+            for (int f = 0; f < n_cur; ++f)
+                for (int j = 0; j < bpf; ++j) {
+                    int t0, t1;
+                    block_span(F, bt, j, &t0, &t1);
+                    double* out = q_pool + (bh * (long)(n_cur * bpf) + (long)f * bpf + j) * D;
+                    for (int d = 0; d < D; ++d) {
+                        double s = 0.0;
+                        for (int t = t0; t < t1; ++t)
+                            s += bf16_to_f64(qh[((long)f * F + t) * D + d]);
+                        out[d] = s / (double)(t1 - t0);
+                    }
+                }
+            /* key blocks and frames */
+            for (int tau = 0; tau < NF; ++tau) {
+                for (int j = 0; j < bpf; ++j) {
+                    int t0, t1;
+                    block_span(F, bt, j, &t0, &t1);
+                    double* out = k_pool + (bh * (long)(NF * bpf) + (long)tau * bpf + j) * D;
+                    for (int d = 0; d < D; ++d) {
+                        double s = 0.0;
+                        for (int t = t0; t < t1; ++t)
+                            s += bf16_to_f64(kh[((long)tau * F + t) * D + d]);
+                        out[d] = s / (double)(t1 - t0);
+                    }
+                }
+                double* fo = k_frame + (bh * NF + tau) * (long)D;
+                for (int d = 0; d < D; ++d) {
+                    double s = 0.0;
+                    for (int t = 0; t < F; ++t)
+                        s += bf16_to_f64(kh[((long)tau * F + t) * D + d]);
+                    fo[d] = s / (double)F;
+                }
+            }
+        }
+}
+
+/* ---- top-k with ties to the lower index ---------------------------------- */
+typedef struct { double score; int idx; } scored;
+
+/* Higher score first; equal scores: lower index first. */
+static int by_score_then_index(const void* pa, const void* pb)
+{
+    const scored* a = (const scored*)pa;
+    const scored* b = (const scored*)pb;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->idx > b->idx) - (a->idx < b->idx);
+}
+
+static int by_int(const void* pa, const void* pb)
+{
+    int a = *(const int*)pa, b = *(const int*)pb;
+    return (a > b) - (a < b);
+}
+
+static double dot(const double* a, const double* b, int D)
+{
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += a[d] * b[d];
+    return s;
+}
+
+/* Number of frames in T_r. */
+int orc_frames_selected(int NF, int n_sink, int n_recent, int n_cur, int chunk_index, int topk_frames)
+{
+    if (chunk_index == 1) return NF;
+    int n_mem = NF - n_sink - n_recent - n_cur;
+    int kf = topk_frames < n_mem ? topk_frames : n_mem;
+    return n_sink + kf + n_recent + n_cur;
+}
+
+/*
+ * [RB] stage 3, first level; [GS] 2.2 "Frame Selection"; [NE] section 3.
+ * For each (b,h,r): p_r(m) = <q~_r, k^_m> for memory frames m; T_r = the sink
+ * frames, the top-k memory frames, the recent frames and the current-chunk frames,
+ * written in ascending frame order to frame_sel[b,h,r, 0..n_sel).
+ * chunk_index == 1 (dense first chunk, [RB] stage 1) selects every frame.
+ * If frame_scores is not NULL it receives p_r(m) as [B,H,Rq,n_mem].
+ */
+void orc_select_frames(int B, int H, int D, int Rq, int NF, int n_sink, int n_recent, int n_cur,
+                       int chunk_index, int topk_frames,
+                       const double* q_pool, const double* k_frame,
+                       int* frame_sel, double* frame_scores)
+{
+    int n_mem = NF - n_sink - n_recent - n_cur;
+    int n_sel = orc_frames_selected(NF, n_sink, n_recent, n_cur, chunk_index, topk_frames);
+    int kf = topk_frames < n_mem ? topk_frames : n_mem;
+    scored* cand = (scored*)malloc(sizeof(scored) * (size_t)(n_mem > 0 ? n_mem : 1));
+    for (long bh = 0; bh < (long)B * H; ++bh)
+        for (int r = 0; r < Rq; ++r) {
+            const double* qr = q_pool + (bh * Rq + r) * (long)D;
+            int* out = frame_sel + (bh * Rq + r) * (long)n_sel;
+            for (int m = 0; m < n_mem; ++m) {
+                cand[m].idx = n_sink + m;
+                cand[m].score = dot(qr, k_frame + (bh * NF + n_sink + m) * (long)D, D);
+                if (frame_scores) frame_scores[(bh * Rq + r) * (long)n_mem + m] = cand[m].score;
+            }
+            if (chunk_index == 1) {
+                for (int t = 0; t < NF; ++t) out[t] = t;
+                continue;
+            }
+            qsort(cand, (size_t)n_mem, sizeof(scored), by_score_then_index);
+            int n = 0;
+            for (int t = 0; t < n_sink; ++t) out[n++] = t;
+            for (int t = 0; t < kf; ++t) out[n++] = cand[t].idx;
+            for (int t = NF - n_recent - n_cur; t < NF; ++t) out[n++] = t;
+            qsort(out, (size_t)n, sizeof(int), by_int);
+        }
+    free(cand);
+}
+
+/*
+ * [RB] stage 3, second level; [GS] 2.2 "Block Selection".
+ * For each (b,h,r) and each tau in T_r: o_r(tau,j) = <q~_r, k~_j^(tau)>,
+ * J_r(tau) = top-k blocks j of frame tau. The mask row is written as the
+ * ascending list of global KV block ids tau*bpf + j with its length in
+ * block_count. chunk_index == 1 keeps every block of every frame.
+ * If block_scores is not NULL it receives o_r(tau, j) as [B,H,Rq,n_sel,bpf].
+ * Returns 0, or -1 if a row would exceed list_cap.
+ */
+int orc_select_blocks(int B, int H, int D, int Rq, int NF, int bpf, int n_sel,
+                      int chunk_index, int topk_blocks,
+                      const double* q_pool, const double* k_pool, const int* frame_sel,
+                      int* block_list, int* block_count, int list_cap, double* block_scores)
+{
+    int kb = (chunk_index == 1 || topk_blocks > bpf) ? bpf : topk_blocks;
+    scored* cand = (scored*)malloc(sizeof(scored) * (size_t)bpf);
+    int* row = (int*)malloc(sizeof(int) * (size_t)(n_sel * bpf + 1));
+    int rc = 0;
+    for (long bh = 0; bh < (long)B * H; ++bh)
+        for (int r = 0; r < Rq; ++r) {
+            const double* qr = q_pool + (bh * Rq + r) * (long)D;
+            const int* T = frame_sel + (bh * Rq + r) * (long)n_sel;
+            int n = 0;
+            for (int s = 0; s < n_sel; ++s) {
+                int tau = T[s];
+                for (int j = 0; j < bpf; ++j) {
+                    cand[j].idx = j;
+                    cand[j].score = dot(qr, k_pool + (bh * (long)NF * bpf + (long)tau * bpf + j) * D, D);
+                    if (block_scores)
+                        block_scores[((bh * Rq + r) * (long)n_sel + s) * bpf + j] = cand[j].score;
+                }
+                qsort(cand, (size_t)bpf, sizeof(scored), by_score_then_index);
+                for (int t = 0; t < kb; ++t) row[n++] = tau * bpf + cand[t].idx;
+            }
+            qsort(row, (size_t)n, sizeof(int), by_int);
+            if (n > list_cap) { rc = -1; n = list_cap; }
+            memcpy(block_list + (bh * Rq + r) * (long)list_cap, row, sizeof(int) * (size_t)n);
+            block_count[bh * Rq + r] = n;
+        }
+    free(row);
+    free(cand);
+    return rc;
+}
+
+/*
+ * [RB] stage 3, last step ("block-sparse attention over the mask").
+ * Softmax attention of query token t of head (b,h) over exactly the valid key
+ * tokens of the blocks listed for t's query block, two-pass (max, then
+ * exp-sum) in fp64:  out = sum_s exp(z_s - max z) v_s / sum_s exp(z_s - max z),
+ * z_s = scale * <q_t, k_s>. rows[i] is a flat query index bh*Lq + t;
+ * out receives [n_rows, D].
+ */
+void orc_attention(int B, int H, int D, int F, int bt, int n_cur, long kv_stride,
+                   const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const int* block_list, const int* block_count, int list_cap,
+                   double scale, const long* rows, long n_rows, double* out)
+{
+    int bpf = ceil_div(F, bt);
+    long Lq = (long)n_cur * F;
+    int Rq = n_cur * bpf;
+    (void)B; (void)H;
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    long max_tok = (long)list_cap * bt;
+    double* z = (double*)malloc(sizeof(double) * (size_t)(max_tok > 0 ? max_tok : 1));
+    long* tok = (long*)malloc(sizeof(long) * (size_t)(max_tok > 0 ? max_tok : 1));
+    for (long i = 0; i < n_rows; ++i) {
+        long bh = rows[i] / Lq;
+        long t = rows[i] % Lq;
+        int r = (int)(t / F) * bpf + (int)((t % F) / bt);
+        for (int d = 0; d < D; ++d) qt[d] = bf16_to_f64(q[(bh * Lq + t) * D + d]);
+        const int* lst = block_list + (bh * Rq + r) * (long)list_cap;
+        int cnt = block_count[bh * Rq + r];
+        /* gather the valid key tokens of the kept blocks */
+        long n = 0;
+        for (int c = 0; c < cnt; ++c) {
+            int g = lst[c];
+            int tau = g / bpf, j = g % bpf;
+            int t0, t1;
+            block_span(F, bt, j, &t0, &t1);
+            for (int s = t0; s < t1; ++s) tok[n++] = (long)tau * F + s;
+        }
+        double* o = out + i * (long)D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (n == 0) continue;
+        const uint16_t* kh = k + bh * kv_stride * D;
+        const uint16_t* vh = v + bh * kv_stride * D;
+        double zmax = -INFINITY;
+        for (long s = 0; s < n; ++s) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += qt[d] * bf16_to_f64(kh[tok[s] * D + d]);
+            z[s] = scale * acc;
+            if (z[s] > zmax) zmax = z[s];
+        }
+        double denom = 0.0;
+        for (long s = 0; s < n; ++s) {
+            double w = exp(z[s] - zmax);
+            denom += w;
+            for (int d = 0; d < D; ++d) o[d] += w * bf16_to_f64(vh[tok[s] * D + d]);
+        }
+        for (int d = 0; d < D; ++d) o[d] /= denom;
+    }
+    free(tok);
+    free(z);
+    free(qt);
+}
+
+/* ---- stage 1: Chunk-Aware Growth ------------------------------------------ */
+/*
+ * [RB] stage 1; [GS] 2.1; [NE] section 2.
+ * s_1 = 0 (first chunk dense); for i > 1, s_i = s_base - alpha_i * beta with
+ * alpha_i = 1 / sqrt(T_i). beta is fixed by the FLOP constraint
+ *     sum_i w_i s_i = s_target * sum_i w_i
+ * (w_i = dense attention FLOPs of chunk i; the sum runs over all chunks when
+ * target_over_all != 0, over chunks 2..n otherwise). The constraint is linear in
+ * beta, so beta = (s_base * sum_{i>1} w_i - s_target * W) / sum_{i>1} w_i alpha_i.
+ * Returns 0, or -1 when the result is infeasible (beta < 0, or some s_i outside
+ * [0, 1), or a non-positive T_i / w_i).
+ */
+int orc_cag(int n_chunks, const double* T, const double* w, double s_base, double s_target,
+            int target_over_all, double* s_out, double* beta_out)
+{
+    if (n_chunks < 2) return -1;
+    double W = 0.0, Wg = 0.0, Wa = 0.0;
+    for (int i = 0; i < n_chunks; ++i) {
+        if (!(T[i] > 0.0) || !(w[i] > 0.0)) return -1;
+        if (i == 0) {
+            if (target_over_all) W += w[i];
+            continue;
+        }
+        double alpha = 1.0 / sqrt(T[i]);
+        W += w[i];
+        Wg += w[i];
+        Wa += w[i] * alpha;
+    }
+    double beta = (s_base * Wg - s_target * W) / Wa;
+    *beta_out = beta;
+    s_out[0] = 0.0;
+    for (int i = 1; i < n_chunks; ++i) s_out[i] = s_base - beta / sqrt(T[i]);
+    if (beta < 0.0) return -1;
+    for (int i = 1; i < n_chunks; ++i)
+        if (s_out[i] < 0.0 || s_out[i] >= 1.0) return -1;
+    return 0;
+}
+
+/*
+ * Per-frame block count for a target block sparsity s: the number of kept
+ * blocks (1 - s) * n_kv_blocks is spread evenly over the n_sel selected frames
+ * and rounded to nearest, clamped to [1, bpf]. The pages give no formula here;
+ * this is the plainest reading of "sparsity" as the dropped fraction of blocks.
+ */
+int orc_blocks_for_sparsity(double s, int n_kv_blocks, int n_sel, int bpf)
+{
+    double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);
+    if (x < 1.0) x = 1.0;
+    if (x > (double)bpf) x = (double)bpf;
+    return (int)x;
+}

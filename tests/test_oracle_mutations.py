@@ -1,0 +1,93 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case copies the oracle's C source to a temporary directory, plants one
+mistake (a dropped term, a wrong sign or index, a wrong divisor), compiles the
+mutant with the same flags, points the oracle binding at it, and checks that at
+least one pin test fails. The real oracle library is never modified.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_attention as t_attn
+import tests.test_oracle_cag as t_cag
+import tests.test_oracle_pool as t_pool
+import tests.test_oracle_select as t_sel
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "lf_oracle.c")
+
+PINS = [
+    t_pool.test_pool_hand_worked,
+    t_pool.test_pool_ramp_closed_form,
+    t_pool.test_pool_constant_and_frame_identity,
+    t_sel.test_select_hand_worked,
+    lambda: [t_sel.test_select_brute_force_with_ties(s) for s in range(6)],
+    lambda: [t_sel.test_select_invariants(*a) for a in [(2, 2, 2), (2, 9, 3), (2, 1, 99), (1, 2, 2)]],
+    lambda: [t_attn.test_all_keep_equals_dense_sdpa(*a) for a in [(100, 64, 16), (64, 64, 8)]],
+    t_attn.test_single_block_and_partial_block,
+    t_attn.test_rows_subset_and_empty_list,
+    t_attn.test_value_is_convex_combination,
+    t_attn.test_per_query_block_lists,
+    t_cag.test_cag_hand_worked,
+    t_cag.test_blocks_for_sparsity_hand_worked,
+    lambda: [t_cag.test_cag_budget_identity_and_growth(s) for s in range(20)],
+]
+
+# (name, text to find, replacement[, how many occurrences; default all]).
+MUTATIONS = [
+    ("partial block mean divides by block size", "out[d] = s / (double)(t1 - t0);", "out[d] = s / (double)bt;"),
+    ("frame mean divides by padded length", "fo[d] = s / (double)F;", "fo[d] = s / (double)(bpf * bt);"),
+    ("blocks straddle frame end", "*t1 = (j + 1) * bt < F ? (j + 1) * bt : F;", "*t1 = (j + 1) * bt;"),
+    ("kv head stride ignored", "const uint16_t* kh = k + bh * kv_stride * D;", "const uint16_t* kh = k + bh * (long)NF * F * D;", 1),
+    ("ties go to the higher index", "return (a->idx > b->idx) - (a->idx < b->idx);", "return (a->idx < b->idx) - (a->idx > b->idx);"),
+    ("bottom-k instead of top-k", "if (a->score > b->score) return -1;", "if (a->score > b->score) return 1;"),
+    ("recent frame dropped", "for (int t = NF - n_recent - n_cur; t < NF; ++t) out[n++] = t;", "for (int t = NF - n_cur; t < NF; ++t) out[n++] = t;"),
+    ("sink frame dropped", "for (int t = 0; t < n_sink; ++t) out[n++] = t;", "for (int t = 1; t < n_sink; ++t) out[n++] = t;"),
+    ("frame scored against a neighbour", "cand[m].score = dot(qr, k_frame + (bh * NF + n_sink + m) * (long)D, D);", "cand[m].score = dot(qr, k_frame + (bh * NF + n_sink + m + 1) * (long)D, D);"),
+    ("block score ignores last dim", "for (int d = 0; d < D; ++d) s += a[d] * b[d];", "for (int d = 0; d + 1 < D; ++d) s += a[d] * b[d];"),
+    ("softmax scale dropped", "z[s] = scale * acc;", "z[s] = acc;"),
+    ("query block index ignores frames", "int r = (int)(t / F) * bpf + (int)((t % F) / bt);", "int r = (int)(t / bt);"),
+    ("softmax denominator dropped", "for (int d = 0; d < D; ++d) o[d] /= denom;", ""),
+    ("CAG sign flipped", "s_out[i] = s_base - beta / sqrt(T[i]);", "s_out[i] = s_base + beta / sqrt(T[i]);"),
+    ("CAG alpha = 1/T", "double alpha = 1.0 / sqrt(T[i]);", "double alpha = 1.0 / T[i];"),
+    ("CAG dense chunk weight dropped", "if (target_over_all) W += w[i];", ""),
+    ("k_b truncates instead of rounding", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel);"),
+]
+
+
+def _build_mutant(tmp_path, find, repl, count=-1):
+    src = open(SRC).read()
+    assert find in src, f"mutation anchor not found: {find}"
+    mutant = src.replace(find, repl, count)
+    c = tmp_path / "mutant.c"
+    c.write_text(mutant)
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math",
+                    "-ffp-contract=off", "-w", "-o", str(so), str(c), "-lm"], check=True)
+    return oracle.configure(ctypes.CDLL(str(so)))
+
+
+def _some_pin_fails():
+    for pin in PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("mutation", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(tmp_path, monkeypatch, mutation):
+    name = mutation[0]
+    lib = _build_mutant(tmp_path, *mutation[1:])
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert _some_pin_fails(), f"no pin caught the planted mistake: {name}"
+
+
+def test_unmutated_copy_passes_all_pins(tmp_path, monkeypatch):
+    lib = _build_mutant(tmp_path, "#include <math.h>", "#include <math.h>")
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert not _some_pin_fails()
