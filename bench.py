@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of one Light Forcing HSA attention call on B200.
+
+A step is one whole HSA call on resident inputs: block/frame mean pooling,
+frame selection, block selection and block-sparse attention (four kernels of
+liblf_hsa.so, called through the C ABI). The default workload is the
+480p-shaped layer call (batch 1, 12 heads, head_dim 128, 1560-token frames,
+21 KV frames = sink + 16 memory + recent + 3-frame current chunk, frame top-4,
+block top-k for 80 % block sparsity), drawn by ``lf_synth``.
+
+Metric: effective TFLOP/s on kept blocks = (4 * valid query rows * valid kept
+key tokens * head_dim, summed over every query block) / time of the whole call.
+The line also carries the microseconds of every kernel, the pooling and
+selection bandwidth, the attention kernel's roofline fraction, the oracle's CPU
+throughput on a bounded sample, and an end-to-end number with host buffers.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torch.distributed.run; each rank runs the same call on
+its own GPU (the call shards by (batch, head) with no exchange: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import platform
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSA µs/call and effective TFLOPS on kept blocks (% bf16 peak); select GB/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="layer480p")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return p.parse_args()
+
+
+def _workload(name):
+    import lf_synth
+    return lf_synth.CONFIGS[name]
+
+
+def _kb(L, shape, w):
+    if w.topk_blocks:
+        return w.topk_blocks
+    n_sel = L.lf_frames_selected(shape, w.chunk_index, w.topk_frames)
+    return L.lf_blocks_for_sparsity(w.sparsity, shape.Nkv, n_sel, shape.bpf)
+
+
+def credited_flops(block_list, block_count, F, bpf, D, n_cur):
+    """4 * valid queries * valid kept keys * D over every query block (host, numpy)."""
+    import numpy as np
+    lst = block_list.reshape(-1, block_list.shape[-1])
+    cnt = block_count.reshape(-1)
+    Rq = n_cur * bpf
+    rem = F - 64 * (bpf - 1)
+    total = 0
+    for row in range(cnt.size):
+        r = row % Rq
+        q_valid = rem if (r % bpf) == bpf - 1 else 64
+        ids = lst[row, :cnt[row]]
+        kv_valid = int(np.where((ids % bpf) == bpf - 1, rem, 64).sum())
+        total += 4 * q_valid * kv_valid * D
+    return float(total)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                clk, cmax, pw = float(parts[0]), float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            mx = cmax
+            if pw > 200.0:  # under load
+                sm.append(clk)
+                for n, flag in zip(names, parts[4:8]):
+                    if flag.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples_under_load": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        return dist, dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
+    return None, 0, 1, 0
+
+
+def _max_over_ranks(dist, x):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _oracle_sample(w, budget_s, q, k, v, block_list=None, block_count=None):
+    """Time the fp64 oracle on a bounded sample of the call; returns a dict with
+    the extrapolated seconds per call and the credited FLOPs of the call."""
+    import numpy as np
+    import oracle
+    s = oracle.shape_of(w)
+    t0 = time.perf_counter()
+    qp, kp, kf = oracle.pool(s, q, k)
+    t_pool = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    sel, _ = oracle.select_frames(s, w.chunk_index, w.topk_frames, qp, kf)
+    n_sel = sel.shape[-1]
+    kb = w.topk_blocks or oracle.blocks_for_sparsity(w.sparsity, s.Nkv, n_sel, s.bpf)
+    lst, cnt, _ = oracle.select_blocks(s, w.chunk_index, kb, qp, kp, sel)
+    t_sel = time.perf_counter() - t0
+    total_rows = s.batch * s.heads * s.Lq
+    rng = np.random.default_rng(0)
+    # grow the attention sample until the budget is spent
+    rows_done, t_att, n = 0, 0.0, 64
+    while t_att < max(0.5, budget_s - t_pool - t_sel) and rows_done < total_rows:
+        rows = rng.integers(0, total_rows, size=n)
+        t0 = time.perf_counter()
+        oracle.attention(s, q, k, v, lst, cnt, rows=rows)
+        t_att += time.perf_counter() - t0
+        rows_done += n
+        n = min(n * 2, 4096)
+    t_call = t_pool + t_sel + t_att * total_rows / rows_done
+    flops = credited_flops(lst, cnt, s.frame_tokens, s.bpf, s.head_dim, s.n_cur)
+    cpu = platform.processor() or platform.machine()
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    cpu = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    sample = (f"fp64 oracle, 1 thread on {cpu} (nproc {os.cpu_count()}): full pooling "
+              f"({t_pool:.2f} s) and selection ({t_sel:.2f} s), attention on {rows_done} of "
+              f"{total_rows} query rows ({t_att:.2f} s) extrapolated linearly to the whole call")
+    return dict(t_call=t_call, flops=flops, sample=sample, wall=t_pool + t_sel + t_att)
+
+
+def run_reference(a):
+    """The oracle as the reference arm: same metric, config and unit."""
+    dist, rank, ws, _ = _dist()
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    import lf_synth
+    w = _workload(a.workload)
+    q, k, v = lf_synth.make_qkv(w)
+    n_steps = a.steps + a.warmup
+    per_step = max(2.0, 150.0 / max(1, n_steps))
+    times = []
+    last = None
+    for i in range(n_steps):
+        r = _oracle_sample(w, per_step, q, k, v)
+        if i >= a.warmup:
+            times.append(r["t_call"])
+        last = r
+    t = statistics.mean(times) if times else last["t_call"]
+    value = last["flops"] / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (lf_synth, seeded; stands in for the pages' VBench 480p rollouts)",
+        "config": _config(w, None),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def _config(w, kb):
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+            "frame_tokens": w.frame_tokens, "kv_frames": w.n_frames,
+            "frames": {"sink": w.n_sink, "memory": w.n_mem, "recent": w.n_recent,
+                       "current": w.n_cur},
+            "q_tokens": w.q_tokens, "kv_tokens": w.kv_tokens, "block_tokens": w.block_tokens,
+            "topk_frames": w.topk_frames, "topk_blocks": kb, "target_sparsity": w.sparsity,
+            "chunk_index": w.chunk_index, "l2": "flushed before every step (512 MiB write)"}
+
+
+def _attn_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if the
+    kernel source has not changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "attn_layer480p_ncu.json")
+    src = os.path.join(ROOT, "block_sparse_attention_lf_b200", "csrc", "lf_attn.cu")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return d.get("dram_bytes_per_launch") if d.get("kernel_src_sha256") == sha else None
+
+
+def run_ours(a):
+    import numpy as np
+    import torch
+
+    dist, rank, ws, local = _dist()
+    torch.cuda.set_device(local)
+    import block_sparse_attention_lf_b200 as L
+    import lf_synth
+
+    w = _workload(a.workload)
+    shape = L.shape_from_workload(w)
+    kb = _kb(L, shape, w)
+    q_h, k_h, v_h = lf_synth.make_qkv(w)
+    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
+    call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb)
+    b = call.buf
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(3, a.warmup)):
+        call(q, k, v)
+    torch.cuda.synchronize()
+    st, detail = L.lf_get_device_error()
+    if st != 0:
+        raise SystemExit(f"device error after warm-up: {st} {detail:#x}")
+    flops = credited_flops(b.block_list.cpu().numpy(), b.block_count.cpu().numpy(),
+                           shape.frame_tokens, shape.bpf, shape.head_dim, shape.n_cur)
+
+    E = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for i in range(a.steps):
+            flush.zero_()
+            e = E[i]
+            e[0].record(stream)
+            call.pool(q, k)
+            e[1].record(stream)
+            L.lf_select_frames(shape, w.chunk_index, w.topk_frames, b.q_pool, b.k_frame, b.frame_sel)
+            e[2].record(stream)
+            L.lf_select_blocks(shape, w.chunk_index, w.topk_frames, kb, b.q_pool, b.k_pool,
+                               b.frame_sel, b.block_list, b.block_count, b.list_cap)
+            e[3].record(stream)
+            call.attend(q, k, v)
+            e[4].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if dist is not None:
+        dist.barrier()
+    st, detail = L.lf_get_device_error()
+    if st != 0:
+        raise SystemExit(f"device error in the timed region: {st} {detail:#x}")
+
+    def mean_ms(i0, i1):
+        return statistics.mean(E[s][i0].elapsed_time(E[s][i1]) for s in range(a.steps))
+
+    t_pool, t_sf, t_sb, t_attn = mean_ms(0, 1), mean_ms(1, 2), mean_ms(2, 3), mean_ms(3, 4)
+    t_step = mean_ms(0, 4)
+    t_step_max = _max_over_ranks(dist, t_step)
+    value = ws * flops / (t_step_max * 1e-3) / 1e12
+
+    # ---- end to end through the public API with pinned host buffers
+    qp_, kp_, vp_ = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    out_h = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    e2e_steps = max(3, min(a.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        q.copy_(qp_, non_blocking=True)
+        k.copy_(kp_, non_blocking=True)
+        v.copy_(vp_, non_blocking=True)
+        call(q, k, v)
+        out_h.copy_(b.out, non_blocking=True)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = _max_over_ranks(dist, statistics.mean(s.elapsed_time(t) for s, t in ev))
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = b.out.numel() * 2
+
+    peaks = _peaks()
+    attn_tflops = flops / (t_attn * 1e-3) / 1e12
+    pool_bytes = (q.numel() + k.numel()) * 2 + (b.q_pool.numel() + b.k_pool.numel() + b.k_frame.numel()) * 4
+    sel_bytes = ((b.q_pool.numel() + b.k_frame.numel() + b.k_pool.numel()) * 4
+                 + (b.frame_sel.numel() + b.block_count.numel()) * 4
+                 + shape.batch * shape.heads * shape.Rq * b.list_cap * 4)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": t_step_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (lf_synth, seeded; stands in for the pages' VBench 480p rollouts)",
+        "config": _config(w, kb),
+        "us_per_call": t_step_max * 1e3,
+        "kernels_us": {"pool": t_pool * 1e3, "select_frames": t_sf * 1e3,
+                       "select_blocks": t_sb * 1e3, "block_sparse_attn": t_attn * 1e3},
+        "kept_tflop_per_call": flops / 1e12,
+        "attn_tflops": attn_tflops,
+        "attn_frac_of_bf16_peak": attn_tflops / peaks["bf16"],
+        "pool_gbs": pool_bytes / (t_pool * 1e-3) / 1e9,
+        "pool_frac_of_hbm": pool_bytes / (t_pool * 1e-3) / 1e9 / peaks["hbm"],
+        "select_gbs": sel_bytes / ((t_sf + t_sb) * 1e-3) / 1e9,
+        "select_over_attn": (t_pool + t_sf + t_sb) / t_attn,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16"],
+                     "traffic": _attn_traffic(),
+                     "peak_source": f"{peaks['source']} bf16 dense burst (MEASURED_PEAKS.json)"},
+        "e2e": {"value": ws * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e},
+        "gpu_launches": 4 * a.steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        r = _oracle_sample(w, a.cpu_budget_s, q_h, k_h, v_h)
+        line["cpu_baseline"] = {"value": r["flops"] / r["t_call"] / 1e12, "unit": "TFLOP/s",
+                                "cores": 1, "kind": "oracle", "sample": r["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,308 @@
+// lf_api.cu -- the C ABI of liblf_hsa.so (declared in include/lf_hsa.h):
+// argument validation, TMA descriptor encoding, kernel launches, the
+// Chunk-Aware Growth solver and the per-device error word.
+#include "lf_hsa.h"
+#include "lf_device.cuh"
+#include "lf_internal.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace {
+
+__device__ int g_device_error;  // first device-side fault code (0 = none)
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+lf_status error_word(int** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return LF_ERR_CUDA;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_err_ptr[dev];
+    return LF_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Derived {
+    int B, H, D, F, bpf, rem, NF, n_sink, n_recent, n_cur, n_mem, Rq, Nkv, Lq, Lkv;
+    long long kv_stride;
+};
+
+lf_status check_shape(const lf_hsa_shape* s, Derived* d)
+{
+    if (!s) return LF_ERR_NULL;
+    if (s->batch < 1 || s->heads < 1) return LF_ERR_SHAPE;
+    if (s->head_dim != 64 && s->head_dim != 128) return LF_ERR_SHAPE;
+    if (s->block_tokens != 64) return LF_ERR_SHAPE;
+    if (s->frame_tokens < 1 || s->frame_tokens > 8192) return LF_ERR_SHAPE;
+    if (s->n_sink < 0 || s->n_recent < 0 || s->n_cur < 1) return LF_ERR_SHAPE;
+    const long long forced = static_cast<long long>(s->n_sink) + s->n_recent + s->n_cur;
+    if (s->n_frames < forced) return LF_ERR_SHAPE;
+    const long long n_mem = s->n_frames - forced;
+    if (n_mem > 1024) return LF_ERR_SHAPE;
+    const long long Lkv = static_cast<long long>(s->n_frames) * s->frame_tokens;
+    const long long stride = s->kv_stride == 0 ? Lkv : s->kv_stride;
+    if (stride < Lkv) return LF_ERR_SHAPE;
+    const long long BH = static_cast<long long>(s->batch) * s->heads;
+    const long long Lq = static_cast<long long>(s->n_cur) * s->frame_tokens;
+    const int bpf = (s->frame_tokens + 63) / 64;
+    // TMA coordinates and kernel indices are 32-bit.
+    if (BH * stride >= (1ll << 31) || BH * Lq >= (1ll << 31)) return LF_ERR_SHAPE;
+    if (BH * s->n_frames * bpf >= (1ll << 31) / 128) return LF_ERR_SHAPE;
+    d->B = s->batch;
+    d->H = s->heads;
+    d->D = s->head_dim;
+    d->F = s->frame_tokens;
+    d->bpf = bpf;
+    d->rem = s->frame_tokens - 64 * (bpf - 1);
+    d->NF = s->n_frames;
+    d->n_sink = s->n_sink;
+    d->n_recent = s->n_recent;
+    d->n_cur = s->n_cur;
+    d->n_mem = static_cast<int>(n_mem);
+    d->Rq = s->n_cur * bpf;
+    d->Nkv = s->n_frames * bpf;
+    d->Lq = static_cast<int>(Lq);
+    d->Lkv = static_cast<int>(Lkv);
+    d->kv_stride = stride;
+    return LF_OK;
+}
+
+int frames_selected(const Derived& d, int chunk_index, int topk_frames)
+{
+    if (chunk_index == 1) return d.NF;
+    const int kf = topk_frames < d.n_mem ? topk_frames : d.n_mem;
+    return d.n_sink + kf + d.n_recent + d.n_cur;
+}
+
+int blocks_per_frame(const Derived& d, int chunk_index, int topk_blocks)
+{
+    if (chunk_index == 1) return d.bpf;
+    return topk_blocks < d.bpf ? topk_blocks : d.bpf;
+}
+
+lf_status launch_status(cudaError_t e) { return e == cudaSuccess ? LF_OK : LF_ERR_CUDA; }
+
+// ---- TMA descriptors ------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 view [rows, D] with a {64, box_rows} box and 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, long long rows, int D, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2u};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lf_version(void) { return "lf_hsa 0.1.0 sm_100a"; }
+
+const char* lf_status_string(lf_status s)
+{
+    switch (s) {
+    case LF_OK: return "ok";
+    case LF_ERR_NULL: return "a required pointer is NULL";
+    case LF_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case LF_ERR_SHAPE: return "unsupported shape";
+    case LF_ERR_TOPK: return "top-k below 1";
+    case LF_ERR_CAP: return "list capacity too small";
+    case LF_ERR_INFEASIBLE: return "chunk-aware growth budget is infeasible";
+    case LF_ERR_CUDA: return "CUDA error";
+    case LF_ERR_DEVICE_TIMEOUT: return "a bounded device wait expired";
+    case LF_ERR_ARG: return "invalid argument";
+    case LF_ERR_LIST: return "block id or count out of range";
+    case LF_ERR_NO_DEVICE: return "no usable CUDA device";
+    }
+    return "unknown status";
+}
+
+int32_t lf_frames_selected(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames)
+{
+    Derived d;
+    if (check_shape(shape, &d) != LF_OK || chunk_index < 1 || topk_frames < 1) return -1;
+    return frames_selected(d, chunk_index, topk_frames);
+}
+
+int32_t lf_list_capacity(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, int32_t topk_blocks)
+{
+    Derived d;
+    if (check_shape(shape, &d) != LF_OK || chunk_index < 1 || topk_frames < 1 || topk_blocks < 1) return -1;
+    return frames_selected(d, chunk_index, topk_frames) * blocks_per_frame(d, chunk_index, topk_blocks);
+}
+
+lf_status lf_pool(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, float* q_pool, float* k_pool,
+                  float* k_frame, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (!q || !k || !q_pool || !k_pool || !k_frame) return LF_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_frame))
+        return LF_ERR_ALIGN;
+    lf::PoolArgs a{q, k, q_pool, k_pool, k_frame, d.B * d.H, d.D, d.F, d.bpf, d.NF, d.n_cur, d.kv_stride};
+    return launch_status(lf::launch_pool(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_select_frames(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, const float* q_pool,
+                           const float* k_frame, int32_t* frame_sel, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (chunk_index < 1) return LF_ERR_ARG;
+    if (topk_frames < 1) return LF_ERR_TOPK;
+    if (!q_pool || !k_frame || !frame_sel) return LF_ERR_NULL;
+    if (!aligned16(q_pool) || !aligned16(k_frame) || !aligned16(frame_sel)) return LF_ERR_ALIGN;
+    lf::SelectFramesArgs a{q_pool, k_frame, frame_sel, d.B * d.H, d.D, d.Rq, d.NF, d.n_sink, d.n_recent,
+                           d.n_cur, frames_selected(d, chunk_index, topk_frames), topk_frames, chunk_index};
+    return launch_status(lf::launch_select_frames(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, int32_t topk_blocks,
+                           const float* q_pool, const float* k_pool, const int32_t* frame_sel, int32_t* block_list,
+                           int32_t* block_count, int32_t list_cap, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (chunk_index < 1) return LF_ERR_ARG;
+    if (topk_frames < 1 || topk_blocks < 1) return LF_ERR_TOPK;
+    if (!q_pool || !k_pool || !frame_sel || !block_list || !block_count) return LF_ERR_NULL;
+    if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(frame_sel) || !aligned16(block_list) ||
+        !aligned16(block_count))
+        return LF_ERR_ALIGN;
+    const int n_sel = frames_selected(d, chunk_index, topk_frames);
+    const int kb = blocks_per_frame(d, chunk_index, topk_blocks);
+    if (list_cap < n_sel * kb) return LF_ERR_CAP;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
+    lf::SelectBlocksArgs a{q_pool, k_pool, frame_sel, block_list, block_count, d.B * d.H, d.D, d.Rq, d.NF,
+                           d.bpf, n_sel, kb, list_cap, chunk_index, err};
+    return launch_status(lf::launch_select_blocks(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const int32_t* block_list, const int32_t* block_count, int32_t list_cap,
+                               float softmax_scale, uint16_t* out, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (list_cap < 0) return LF_ERR_CAP;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return LF_ERR_ARG;
+    if (!q || !k || !v || !block_list || !block_count || !out) return LF_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_list) || !aligned16(block_count) ||
+        !aligned16(out))
+        return LF_ERR_ALIGN;
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LF_ERR_NO_DEVICE;
+    if (major != 10 || minor != 0) return LF_ERR_NO_DEVICE;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d.D));
+    const long long BH = static_cast<long long>(d.B) * d.H;
+    lf::AttnMaps m;
+    const long long q_rows = BH * d.Lq, kv_rows = BH * d.kv_stride;
+    if (!encode_rows(&m.q, q, q_rows, d.D, 64) || !encode_rows(&m.q_rem, q, q_rows, d.D, d.rem) ||
+        !encode_rows(&m.k, k, kv_rows, d.D, 64) || !encode_rows(&m.k_rem, k, kv_rows, d.D, d.rem) ||
+        !encode_rows(&m.v, v, kv_rows, d.D, 64) || !encode_rows(&m.v_rem, v, kv_rows, d.D, d.rem))
+        return LF_ERR_CUDA;
+    lf::AttnArgs a{block_list, block_count, out, list_cap, d.Rq, d.bpf, d.F, d.Lq, d.Nkv, d.rem, d.kv_stride,
+                   scale * 1.4426950408889634f, err};
+    return launch_status(lf::launch_attn(m, a, d.D, static_cast<int>(BH * d.Rq), static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_cag_budget(int32_t n_chunks, const double* T, const double* flops_w, double s_base, double s_target,
+                        int32_t target_over_all, double* s_out, double* beta_out)
+{
+    if (!T || !s_out || !beta_out) return LF_ERR_NULL;
+    if (n_chunks < 2) return LF_ERR_ARG;
+    if (!(s_base >= 0.0 && s_base < 1.0) || !(s_target >= 0.0 && s_target < 1.0)) return LF_ERR_ARG;
+    double W = 0.0, Wg = 0.0, Wa = 0.0;
+    for (int i = 0; i < n_chunks; ++i) {
+        const double w = flops_w ? flops_w[i] : static_cast<double>(i + 1);
+        if (!(T[i] > 0.0) || !(w > 0.0) || std::isinf(T[i]) || std::isinf(w)) return LF_ERR_ARG;
+        if (i == 0) {
+            if (target_over_all) W += w;  // the dense first chunk counts in the budget
+            continue;
+        }
+        const double alpha = 1.0 / std::sqrt(T[i]);
+        W += w;
+        Wg += w;
+        Wa += w * alpha;
+    }
+    // sum_{i>1} w_i (s_base - alpha_i beta) = s_target * W, linear in beta.
+    const double beta = (s_base * Wg - s_target * W) / Wa;
+    *beta_out = beta;
+    s_out[0] = 0.0;
+    bool feasible = beta >= 0.0;
+    for (int i = 1; i < n_chunks; ++i) {
+        s_out[i] = s_base - beta / std::sqrt(T[i]);
+        if (!(s_out[i] >= 0.0 && s_out[i] < 1.0)) feasible = false;
+    }
+    return feasible ? LF_OK : LF_ERR_INFEASIBLE;
+}
+
+int32_t lf_blocks_for_sparsity(double s, int32_t n_kv_blocks, int32_t n_sel_frames, int32_t bpf)
+{
+    if (!(s >= 0.0 && s < 1.0) || n_kv_blocks < 1 || n_sel_frames < 1 || bpf < 1) return -1;
+    double x = std::floor((1.0 - s) * static_cast<double>(n_kv_blocks) / static_cast<double>(n_sel_frames) + 0.5);
+    if (x < 1.0) x = 1.0;
+    if (x > static_cast<double>(bpf)) x = static_cast<double>(bpf);
+    return static_cast<int32_t>(x);
+}
+
+lf_status lf_get_device_error(int32_t* detail)
+{
+    int* p = nullptr;
+    lf_status st = error_word(&p);
+    if (st != LF_OK) return st;
+    int h = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LF_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof h) != cudaSuccess) return LF_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return LF_ERR_CUDA;
+    if (detail) *detail = h;
+    if (h == 0) return LF_OK;
+    return (h & lf::DEVERR_TIMEOUT) ? LF_ERR_DEVICE_TIMEOUT : LF_ERR_LIST;
+}
+
+}  // extern "C"

@@ -1,0 +1,446 @@
+// lf_attn.cu -- block-sparse softmax attention of one HSA call on sm_100a
+// tensor cores ("Light Forcing：通过稀疏注意力加速自回归视频扩散",
+// paper.rainbus.top, execution flow, stage 3, final step: attention computed
+// only over the kept (frame, block) pairs of B_r).
+//
+// Design (B200-first; the pages' kernel is prior art only):
+//   * One CTA per query block (64 query tokens of one head, its own KV block
+//     list). CTAs are ordered head-major so a head's K/V stay L2-resident while
+//     its query blocks run.
+//   * KV-major formulation. A tile is two listed KV blocks (128 tokens). The
+//     tensor core computes S^T = K_tile * Q^T (M = 128 KV tokens, N = 64
+//     queries, K = head_dim) into TMEM, and O^T += V_tile^T * P^T (M = 128
+//     head-dim rows, N = 64 queries, K = 128 KV tokens). Both MMAs therefore
+//     run with M = 128 on exactly the listed blocks, with no union of
+//     neighbouring query blocks' lists.
+//   * Warp roles (320 threads): warp 0 issues TMA loads (Q once; per tile the
+//     listed K and V blocks, 64-row boxes, 128-byte swizzle), warp 1 allocates
+//     TMEM and issues tcgen05.mma from one thread, warps 2-9 are two softmax
+//     warpgroups. TMEM lane t of S^T is KV token t of the tile, so each
+//     softmax thread owns one KV token and 32 query columns (warpgroup 0:
+//     queries 0-31, warpgroup 1: queries 32-63).
+//   * Online softmax in fp32, base 2, with a lazy stabiliser: each query
+//     column keeps m (running max of scale*log2(e)*score); a tile whose scores
+//     stay within m + 8 (p <= 256) is exponentiated against the current m with
+//     no cross-thread work; only when some score exceeds that bound does the
+//     warpgroup compute the exact column maxima of the tile (butterfly
+//     reductions + shared memory) and rescale its columns of O^T in TMEM. Row
+//     sums are kept per thread and reduced once at the end.
+//   * P^T goes to shared memory as bf16 in the 128-byte-swizzled MN-major
+//     layout the MMA reads; masked KV tokens (past the end of a partial block,
+//     or the unused half of an odd last tile) get P = 0.
+//   * Pipelines: K ring of 2 slots, V ring of 3, S double-buffered in TMEM, P
+//     double-buffered in shared memory; the MMA thread issues S for tile i+2
+//     right after PV for tile i, so S is ready before the softmax needs it.
+//   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
+//     flag and the device error word, every role runs its remaining steps
+//     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
+//     and the kernel returns.
+#include "lf_device.cuh"
+#include "lf_internal.h"
+
+#include <cuda_bf16.h>
+
+namespace lf {
+namespace {
+
+constexpr int ATTN_THREADS = 320;
+constexpr int KSLOTS = 2;
+constexpr int VSLOTS = 3;
+constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
+constexpr uint32_t TMEM_COLS = 256;         // S0: 0-63, S1: 64-127, O^T: 128-191
+
+template <int D>
+struct AttnLayout {
+    static constexpr int NP = D / 64;                       // 64-element panels of head_dim
+    static constexpr uint32_t PANEL_Q = 64u * 128u;          // 64 rows x 128 B
+    static constexpr uint32_t PANEL_KV = 128u * 128u;        // 128 rows x 128 B
+    static constexpr uint32_t Q_BYTES = NP * PANEL_Q;
+    static constexpr uint32_t K_SLOT = NP * PANEL_KV;
+    static constexpr uint32_t V_SLOT = 2u * PANEL_KV;        // always 2 panels: the PV MMA has M = 128
+    static constexpr uint32_t P_BUF = 128u * 128u;           // P^T: 128 KV rows x 64 queries bf16
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + KSLOTS * K_SLOT;
+    static constexpr uint32_t OFF_P = OFF_V + VSLOTS * V_SLOT;
+    static constexpr uint32_t OFF_AUX = OFF_P + 2u * P_BUF;
+};
+
+struct AttnAux {
+    uint64_t q_full;
+    uint64_t k_full[KSLOTS], k_empty[KSLOTS];
+    uint64_t v_full[VSLOTS], v_empty[VSLOTS];
+    uint64_t s_full[2], p_full[2], p_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    float red[2][4][32];
+};
+
+template <int D>
+constexpr uint32_t attn_smem_bytes()
+{
+    return AttnLayout<D>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux)) + 1024u;
+}
+
+template <bool MAX>
+__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = upper ? v[i] : v[i + s];
+            const float keep = upper ? v[i + s] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, s);
+            v[i] = MAX ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+}
+
+// Token rows of KV block g (0 when g is not a valid block id) and its first
+// row in the flattened [B*H*kv_stride, D] view of k / v.
+__device__ __forceinline__ int block_rows(const AttnArgs& a, int g, int bh, int* first_row)
+{
+    if (g < 0 || g >= a.Nkv) return 0;
+    const int tau = g / a.bpf;
+    const int j = g - tau * a.bpf;
+    *first_row = static_cast<int>(static_cast<long long>(bh) * a.kv_stride + static_cast<long long>(tau) * a.F + j * 64);
+    return (j == a.bpf - 1) ? a.rem : 64;
+}
+
+template <int D>
+__global__ void __launch_bounds__(ATTN_THREADS, 1)
+attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rem,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k_rem,
+            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_v_rem,
+            const AttnArgs a)
+{
+    using L = AttnLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    AttnAux& x = *reinterpret_cast<AttnAux*>(smem + L::OFF_AUX);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = blockIdx.x;
+    const int bh = row / a.Rq;
+    const int r = row - bh * a.Rq;
+    int cnt = __ldg(a.block_count + row);
+    if (cnt < 0 || cnt > a.list_cap) {
+        if (tid == 0) record_error(a.err, DEVERR_LIST | 1);
+        cnt = cnt < 0 ? 0 : a.list_cap;
+    }
+    const int* lst = a.block_list + static_cast<long long>(row) * a.list_cap;
+    const int n_tiles = (cnt + 1) >> 1;
+    const int fq = r / a.bpf;
+    const int jq = r - fq * a.bpf;
+    const int q_rows = (jq == a.bpf - 1) ? a.rem : 64;
+    const int q_row0 = bh * a.Lq + fq * a.F + jq * 64;
+
+    if (tid == 0) {
+        mbar_init(&x.q_full, 1);
+        for (int s = 0; s < KSLOTS; ++s) { mbar_init(&x.k_full[s], 1); mbar_init(&x.k_empty[s], 1); }
+        for (int s = 0; s < VSLOTS; ++s) { mbar_init(&x.v_full[s], 1); mbar_init(&x.v_empty[s], 1); }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&x.s_full[s], 1);
+            mbar_init(&x.p_full[s], 256);
+            mbar_init(&x.p_empty[s], 1);
+        }
+        mbar_init(&x.drain, 1);
+        x.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&x.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    // V slots are read in full by the PV MMA (M = 128 head-dim rows, K = 128
+    // KV rows) even where a tile loads fewer rows; they start at zero so those
+    // rows are finite (P is zero there). Q rows past a partial query block
+    // only feed discarded output columns; zero them as well.
+    {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        uint4* vz = reinterpret_cast<uint4*>(smem + L::OFF_V);
+        for (int i = tid; i < static_cast<int>(VSLOTS * L::V_SLOT / 16); i += ATTN_THREADS) vz[i] = z;
+        if (q_rows < 64) {
+            uint4* qz = reinterpret_cast<uint4*>(smem + L::OFF_Q);
+            for (int i = tid; i < static_cast<int>(L::Q_BYTES / 16); i += ATTN_THREADS) qz[i] = z;
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = x.tmem_base;
+    volatile int* abort_flag = &x.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
+            mbar_arrive_expect_tx(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
+            for (int p = 0; p < L::NP; ++p)
+                tma_load_2d(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
+            int k_armed = 0, v_armed = 0;  // tiles whose loads were issued
+            for (int i = 0; i < n_tiles; ++i) {
+                const int nb = min(2, cnt - 2 * i);
+                int rows[2] = {0, 0}, first[2] = {0, 0};
+                for (int h = 0; h < nb; ++h) {
+                    const int g = __ldg(lst + 2 * i + h);
+                    rows[h] = block_rows(a, g, bh, &first[h]);
+                    if (rows[h] == 0) record_error(a.err, DEVERR_LIST | 2);
+                }
+                const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NP);
+                const int ks = i % KSLOTS;
+                if (!mbar_wait(&x.k_empty[ks], ((i / KSLOTS) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
+                if (bytes) mbar_arrive_expect_tx(&x.k_full[ks], bytes);
+                else mbar_arrive(&x.k_full[ks]);
+                for (int h = 0; h < nb; ++h) {
+                    if (!rows[h]) continue;
+                    const CUtensorMap* m = rows[h] == 64 ? &tm_k : &tm_k_rem;
+                    for (int p = 0; p < L::NP; ++p)
+                        tma_load_2d(smem + L::OFF_K + ks * L::K_SLOT + p * L::PANEL_KV + h * 64 * 128, m,
+                                    p * 64, first[h], &x.k_full[ks]);
+                }
+                k_armed = i + 1;
+                const int vs = i % VSLOTS;
+                if (!mbar_wait(&x.v_empty[vs], ((i / VSLOTS) & 1) ^ 1, abort_flag, a.err, 0x11)) break;
+                if (bytes) mbar_arrive_expect_tx(&x.v_full[vs], bytes);
+                else mbar_arrive(&x.v_full[vs]);
+                for (int h = 0; h < nb; ++h) {
+                    if (!rows[h]) continue;
+                    const CUtensorMap* m = rows[h] == 64 ? &tm_v : &tm_v_rem;
+                    for (int p = 0; p < L::NP; ++p)
+                        tma_load_2d(smem + L::OFF_V + vs * L::V_SLOT + p * L::PANEL_KV + h * 64 * 128, m,
+                                    p * 64, first[h], &x.v_full[vs]);
+                }
+                v_armed = i + 1;
+            }
+            if (*abort_flag) {
+                // Let every copy already issued land before the CTA exits.
+                mbar_drain(&x.q_full, 0, 10000000ull);
+                for (int i = max(0, k_armed - KSLOTS); i < k_armed; ++i)
+                    mbar_drain(&x.k_full[i % KSLOTS], (i / KSLOTS) & 1, 10000000ull);
+                for (int i = max(0, v_armed - VSLOTS); i < v_armed; ++i)
+                    mbar_drain(&x.v_full[i % VSLOTS], (i / VSLOTS) & 1, 10000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, true);
+            const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+            const uint32_t sK = smem_u32(smem + L::OFF_K);
+            const uint32_t sV = smem_u32(smem + L::OFF_V);
+            const uint32_t sP = smem_u32(smem + L::OFF_P);
+            bool issued_any = false;
+            bool ok = mbar_wait(&x.q_full, 0, abort_flag, a.err, 0x20);
+            auto issue_s = [&](int j) -> bool {
+                const int ks = j % KSLOTS;
+                if (!mbar_wait(&x.k_full[ks], (j / KSLOTS) & 1, abort_flag, a.err, 0x21)) return false;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>((j & 1) * 64);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t panel = static_cast<uint32_t>(kk >> 2);
+                    const uint64_t ad = sdesc_sw128(sK + ks * L::K_SLOT + panel * L::PANEL_KV + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
+                    umma_bf16(d, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&x.k_empty[ks]);
+                umma_commit(&x.s_full[j & 1]);
+                issued_any = true;
+                return true;
+            };
+            if (ok && n_tiles > 0) ok = issue_s(0);
+            if (ok && n_tiles > 1) ok = issue_s(1);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                if (!mbar_wait(&x.p_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x22)) break;
+                const int vs = i % VSLOTS;
+                if (!mbar_wait(&x.v_full[vs], (i / VSLOTS) & 1, abort_flag, a.err, 0x23)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // A = V^T (M = head_dim, MN-major: 64-wide panels LBO apart, 8-row K groups SBO apart)
+                    const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * 2048, L::PANEL_KV, 1024);
+                    // B = P^T (N = 64 queries, MN-major, one 64-wide panel)
+                    const uint64_t bd = sdesc_sw128(sP + (i & 1) * L::P_BUF + kk * 2048, L::P_BUF, 1024);
+                    umma_bf16(tmem + 128, ad, bd, IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&x.v_empty[vs]);
+                umma_commit(&x.p_empty[i & 1]);
+                issued_any = true;
+                if (i + 2 < n_tiles && !issue_s(i + 2)) break;
+            }
+            if (*abort_flag && issued_any) {
+                umma_commit(&x.drain);
+                mbar_drain(&x.drain, 0, 10000000ull);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int wg = (warp - 2) >> 2;        // query columns [32*wg, 32*wg + 32)
+        const int sp = warp & 3;               // TMEM sub-partition of this warp
+        const int t = sp * 32 + lane;          // KV token of the tile / head-dim row of O^T
+        const int bar_id = 1 + wg;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
+        const uint32_t col0 = static_cast<uint32_t>(wg * 32);
+        const float sl2 = a.scale_log2;
+        float m[32], l[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) { m[c] = -INFINITY; l[c] = 0.f; }
+
+        for (int i = 0; i < n_tiles; ++i) {
+            const int hb = t >> 6;
+            const int bi = 2 * i + hb;
+            bool valid = false;
+            if (bi < cnt) {
+                int first;
+                const int rows = block_rows(a, __ldg(lst + bi), bh, &first);
+                valid = (t & 63) < rows;
+            }
+            mbar_wait(&x.s_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x30);
+            __syncwarp();
+            tc_fence_after();
+            float s[32];
+            tmem_ld32(lane_base + static_cast<uint32_t>((i & 1) * 64) + col0, s);
+            tmem_ld_wait();
+            float xmax = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                s[c] = valid ? s[c] * sl2 : -INFINITY;
+                xmax = fmaxf(xmax, s[c] - m[c]);
+            }
+            const bool need = named_bar_or(bar_id, 128, xmax > LAZY_RESCALE_LOG2);
+            if (need) {
+                float v[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] = s[c];
+                transpose_reduce<true>(v, lane);
+                x.red[wg][sp][lane] = v[0];
+                named_bar_sync(bar_id, 128);
+                float alpha[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float tmax = fmaxf(fmaxf(x.red[wg][0][c], x.red[wg][1][c]),
+                                             fmaxf(x.red[wg][2][c], x.red[wg][3][c]));
+                    const float mn = fmaxf(m[c], tmax);
+                    alpha[c] = (mn == -INFINITY) ? 1.f : fast_exp2(m[c] - mn);
+                    m[c] = mn;
+                    l[c] *= alpha[c];
+                }
+                named_bar_sync(bar_id, 128);
+                if (i > 0) {
+                    // O^T columns of this warpgroup hold PV_0..PV_{i-1}: wait for
+                    // PV_{i-2} (other P buffer) and PV_{i-1}, then rescale.
+                    mbar_wait(&x.p_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag, a.err, 0x31);
+                    mbar_wait(&x.p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.err, 0x32);
+                    __syncwarp();
+                    tc_fence_after();
+                    float o[32];
+                    tmem_ld32(lane_base + 128u + col0, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] *= alpha[c];
+                    tmem_st32(lane_base + 128u + col0, o);
+                    tmem_st_wait();
+                }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+                const float p0 = valid ? fast_exp2(s[c] - m[c]) : 0.f;
+                const float p1 = valid ? fast_exp2(s[c + 1] - m[c + 1]) : 0.f;
+                l[c] += p0;
+                l[c + 1] += p1;
+                pk[c >> 1] = pack_bf16x2(p0, p1);
+            }
+            // P buffer (i & 1) was last read by PV_{i-2}.
+            if (i >= 2) mbar_wait(&x.p_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag, a.err, 0x33);
+            __syncwarp();
+            uint8_t* prow = smem + L::OFF_P + (i & 1) * L::P_BUF + (t >> 3) * 1024 + (t & 7) * 128;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int chunk = (wg * 4 + k) ^ (t & 7);
+                *reinterpret_cast<uint4*>(prow + chunk * 16) =
+                    make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&x.p_full[i & 1]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        if (n_tiles > 0)
+            mbar_wait(&x.p_empty[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, a.err, 0x34);
+        __syncwarp();
+        tc_fence_after();
+        transpose_reduce<false>(l, lane);
+        x.red[wg][sp][lane] = l[0];
+        named_bar_sync(bar_id, 128);
+        float o[32];
+        if (n_tiles > 0) {
+            tmem_ld32(lane_base + 128u + col0, o);
+            tmem_ld_wait();
+        } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        // Stage O (bf16, [query][head_dim]) in the K ring, free now.
+        __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K);
+        if (t < D) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float lsum = x.red[wg][0][c] + x.red[wg][1][c] + x.red[wg][2][c] + x.red[wg][3][c];
+                const float val = lsum > 0.f ? o[c] / lsum : 0.f;
+                ostage[(col0 + c) * D + t] = __float2bfloat16_rn(val);
+            }
+        }
+        named_bar_sync(3, 256);
+        const int chunks = q_rows * (D / 8);
+        for (int idx = tid - 64; idx < chunks; idx += 256) {
+            const int qq = idx / (D / 8);
+            const int c8 = idx - qq * (D / 8);
+            *reinterpret_cast<uint4*>(a.out + (static_cast<long long>(q_row0) + qq) * D + c8 * 8) =
+                *reinterpret_cast<const uint4*>(ostage + qq * D + c8 * 8);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int D>
+cudaError_t launch_attn_d(const AttnMaps& m, const AttnArgs& a, int n_rows, cudaStream_t s)
+{
+    constexpr uint32_t smem = attn_smem_bytes<D>();
+    static int configured_device = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    attn_kernel<D><<<static_cast<unsigned>(n_rows), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v, m.v_rem, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, int n_rows, cudaStream_t s)
+{
+    if (n_rows <= 0) return cudaSuccess;
+    return D == 128 ? launch_attn_d<128>(m, a, n_rows, s) : launch_attn_d<64>(m, a, n_rows, s);
+}
+
+}  // namespace lf

@@ -1,0 +1,57 @@
+// lf_internal.h -- launch interfaces between the C ABI layer (lf_api.cu) and
+// the kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace lf {
+
+struct PoolArgs {
+    const uint16_t* q;
+    const uint16_t* k;
+    float* q_pool;
+    float* k_pool;
+    float* k_frame;
+    int BH, D, F, bpf, NF, n_cur;
+    long long kv_stride;  // tokens between heads in k
+};
+
+struct SelectFramesArgs {
+    const float* q_pool;
+    const float* k_frame;
+    int* frame_sel;
+    int BH, D, Rq, NF, n_sink, n_recent, n_cur, n_sel, topk, chunk_index;
+};
+
+struct SelectBlocksArgs {
+    const float* q_pool;
+    const float* k_pool;
+    const int* frame_sel;
+    int* block_list;
+    int* block_count;
+    int BH, D, Rq, NF, bpf, n_sel, kb, list_cap, chunk_index;
+    int* err;
+};
+
+struct AttnArgs {
+    const int* block_list;
+    const int* block_count;
+    uint16_t* out;
+    int list_cap, Rq, bpf, F, Lq, Nkv, rem;
+    long long kv_stride;
+    float scale_log2;  // softmax scale * log2(e)
+    int* err;
+};
+
+struct AttnMaps {
+    CUtensorMap q, q_rem, k, k_rem, v, v_rem;
+};
+
+cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
+cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s);
+cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s);
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, int n_rows, cudaStream_t s);
+
+}  // namespace lf

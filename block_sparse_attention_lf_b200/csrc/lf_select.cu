@@ -1,0 +1,251 @@
+// lf_select.cu -- two-level mask selection of one HSA call ("Light Forcing：通过
+// 稀疏注意力加速自回归视频扩散", paper.rainbus.top, execution flow, stage 3:
+// frame scores p_r = <q~_r, k^_M> and top-k frames T_r with the sink, most
+// recent and current-chunk frames always kept; block scores
+// o_r(tau,j) = <q~_r, k~_j^(tau)> and top-k blocks J_r(tau) in each selected
+// frame, giving the mask B_r(tau,j) = 1[tau in T_r, j in J_r(tau)];
+// gist.science Technical Summary 2.2 "Two-Level Mask Selection").
+//
+// Latency-bound (a few MB of pooled fp32 data, read from L2). One warp per
+// scored row:
+//   * scores: each lane holds head_dim/32 coordinates of q~_r; for a group of
+//     32 candidates each lane forms its 32 partial products and a butterfly
+//     "transpose reduce" (31 shuffles) leaves candidate c's full inner product
+//     in lane c;
+//   * ranking: a candidate is the 64-bit key (orderable(score) << 32) |
+//     (0xFFFFFFFF - index), so a larger key is a larger score, and among equal
+//     scores the lower index; keys are unique.
+//   * frames: top-k by k rounds of warp arg-max over the keys;
+//   * blocks: top-k by rank counting (rank = number of larger keys), then a
+//     ballot/popc compaction writes the kept block ids in ascending order.
+#include "lf_device.cuh"
+#include "lf_internal.h"
+
+namespace lf {
+namespace {
+
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
+
+// After the call lane c holds sum over lanes of v[c] in v[0].
+__device__ __forceinline__ void transpose_reduce_sum(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = upper ? v[i] : v[i + s];
+            const float keep = upper ? v[i + s] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+        }
+    }
+}
+
+template <int EPL>
+__device__ __forceinline__ void load_lane(float (&dst)[EPL], const float* p)
+{
+    if constexpr (EPL == 4) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(p));
+        dst[0] = t.x; dst[1] = t.y; dst[2] = t.z; dst[3] = t.w;
+    } else {
+        const float2 t = __ldg(reinterpret_cast<const float2*>(p));
+        dst[0] = t.x; dst[1] = t.y;
+    }
+}
+
+// Scores of candidates base..base+31 (rows of `rows`, D floats each, only the
+// first n are real); returns the score of candidate base+lane (0 if beyond n).
+template <int D>
+__device__ __forceinline__ float score_group(const float (&qv)[D / 32], const float* rows, int base,
+                                             int n, int lane)
+{
+    constexpr int EPL = D / 32;
+    float part[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        part[c] = 0.f;
+        if (base + c < n) {
+            float kv[EPL];
+            load_lane<EPL>(kv, rows + static_cast<long long>(base + c) * D + lane * EPL);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) part[c] = fmaf(qv[e], kv[e], part[c]);
+        }
+    }
+    transpose_reduce_sum(part, lane);
+    return part[0];
+}
+
+__device__ __forceinline__ uint64_t make_key(float score, int idx)
+{
+    return (static_cast<uint64_t>(orderable(score)) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v)
+{
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = o > v ? o : v;
+    }
+    return v;
+}
+
+// KPL = key slots per lane = ceil(n_mem / 32).
+template <int D, int KPL>
+__global__ void __launch_bounds__(SEL_THREADS) select_frames_kernel(const SelectFramesArgs a)
+{
+    constexpr int EPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
+    if (row >= static_cast<long long>(a.BH) * a.Rq) return;
+    int* out = a.frame_sel + row * a.n_sel;
+    if (a.chunk_index == 1) {
+        for (int t = lane; t < a.NF; t += 32) out[t] = t;
+        return;
+    }
+    const int bh = static_cast<int>(row / a.Rq);
+    const int n_mem = a.NF - a.n_sink - a.n_recent - a.n_cur;
+    const int kf = a.topk < n_mem ? a.topk : n_mem;
+
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    const float* kmem = a.k_frame + (static_cast<long long>(bh) * a.NF + a.n_sink) * D;
+
+    uint64_t key[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const float sc = score_group<D>(qv, kmem, i * 32, n_mem, lane);
+        const int m = i * 32 + lane;
+        key[i] = (m < n_mem) ? make_key(sc, m) : 0ull;
+    }
+
+    uint32_t sel = 0;  // bit i: key slot i of this lane is in the top-k
+    for (int t = 0; t < kf; ++t) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) best = key[i] > best ? key[i] : best;
+        const uint64_t wbest = warp_max_u64(best);
+#pragma unroll
+        for (int i = 0; i < KPL; ++i)
+            if (key[i] == wbest && wbest != 0ull) {
+                sel |= 1u << i;
+                key[i] = 0ull;
+            }
+    }
+
+    // T_r = sinks, selected memory frames (ascending), recent + current frames.
+    for (int t = lane; t < a.n_sink; t += 32) out[t] = t;
+    int prefix = a.n_sink;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const bool s = (sel >> i) & 1u;
+        const uint32_t mask = __ballot_sync(0xffffffffu, s);
+        if (s) out[prefix + __popc(mask & lt)] = a.n_sink + i * 32 + lane;
+        prefix += __popc(mask);
+    }
+    const int tail0 = a.NF - a.n_recent - a.n_cur;
+    for (int t = lane; t < a.n_recent + a.n_cur; t += 32) out[a.n_sink + kf + t] = tail0 + t;
+}
+
+// One warp per (row, selected-frame slot). KPL = ceil(bpf / 32).
+template <int D, int KPL>
+__global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const SelectBlocksArgs a)
+{
+    constexpr int EPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long gw = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
+    if (gw >= static_cast<long long>(a.BH) * a.Rq * a.n_sel) return;
+    const long long row = gw / a.n_sel;
+    const int s = static_cast<int>(gw - row * a.n_sel);
+    const int bh = static_cast<int>(row / a.Rq);
+    int* out = a.block_list + row * a.list_cap + static_cast<long long>(s) * a.kb;
+    if (s == 0 && lane == 0) a.block_count[row] = a.n_sel * a.kb;
+
+    const int tau = (a.chunk_index == 1) ? s : __ldg(a.frame_sel + row * a.n_sel + s);
+    if (tau < 0 || tau >= a.NF) {
+        // A frame id outside the call: write ids the attention kernel rejects.
+        for (int t = lane; t < a.kb; t += 32) out[t] = -1;
+        if (lane == 0) record_error(a.err, DEVERR_LIST | 3);
+        return;
+    }
+
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    const float* kblk = a.k_pool + (static_cast<long long>(bh) * a.NF * a.bpf + static_cast<long long>(tau) * a.bpf) * D;
+
+    uint64_t key[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const float sc = score_group<D>(qv, kblk, i * 32, a.bpf, lane);
+        const int j = i * 32 + lane;
+        key[i] = (j < a.bpf) ? make_key(sc, j) : 0ull;
+    }
+
+    int rank[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) rank[i] = 0;
+    for (int src = 0; src < 32; ++src) {
+#pragma unroll
+        for (int i2 = 0; i2 < KPL; ++i2) {
+            const uint64_t o = __shfl_sync(0xffffffffu, key[i2], src);
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) rank[i] += (o > key[i]) ? 1 : 0;
+        }
+    }
+
+    int prefix = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const bool keep = key[i] != 0ull && rank[i] < a.kb;
+        const uint32_t mask = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[prefix + __popc(mask & lt)] = tau * a.bpf + i * 32 + lane;
+        prefix += __popc(mask);
+    }
+}
+
+template <int D>
+cudaError_t launch_frames_d(const SelectFramesArgs& a, unsigned grid, cudaStream_t s)
+{
+    const int n_mem = a.NF - a.n_sink - a.n_recent - a.n_cur;
+    const int kpl = (n_mem + 31) / 32;
+    if (a.chunk_index == 1 || kpl <= 1) select_frames_kernel<D, 1><<<grid, SEL_THREADS, 0, s>>>(a);
+    else if (kpl <= 2) select_frames_kernel<D, 2><<<grid, SEL_THREADS, 0, s>>>(a);
+    else if (kpl <= 4) select_frames_kernel<D, 4><<<grid, SEL_THREADS, 0, s>>>(a);
+    else if (kpl <= 8) select_frames_kernel<D, 8><<<grid, SEL_THREADS, 0, s>>>(a);
+    else if (kpl <= 16) select_frames_kernel<D, 16><<<grid, SEL_THREADS, 0, s>>>(a);
+    else select_frames_kernel<D, 32><<<grid, SEL_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_blocks_d(const SelectBlocksArgs& a, unsigned grid, cudaStream_t s)
+{
+    const int kpl = (a.bpf + 31) / 32;
+    if (kpl <= 1) select_blocks_kernel<D, 1><<<grid, SEL_THREADS, 0, s>>>(a);
+    else if (kpl <= 2) select_blocks_kernel<D, 2><<<grid, SEL_THREADS, 0, s>>>(a);
+    else select_blocks_kernel<D, 4><<<grid, SEL_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s)
+{
+    const long long rows = static_cast<long long>(a.BH) * a.Rq;
+    if (rows <= 0) return cudaSuccess;
+    const unsigned grid = static_cast<unsigned>((rows + SEL_WARPS - 1) / SEL_WARPS);
+    return a.D == 128 ? launch_frames_d<128>(a, grid, s) : launch_frames_d<64>(a, grid, s);
+}
+
+cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s)
+{
+    const long long warps = static_cast<long long>(a.BH) * a.Rq * a.n_sel;
+    if (warps <= 0) return cudaSuccess;
+    const unsigned grid = static_cast<unsigned>((warps + SEL_WARPS - 1) / SEL_WARPS);
+    return a.D == 128 ? launch_blocks_d<128>(a, grid, s) : launch_blocks_d<64>(a, grid, s);
+}
+
+}  // namespace lf

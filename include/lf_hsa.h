@@ -1,0 +1,225 @@
+/*
+ * lf_hsa.h -- C ABI of the B200 (sm_100a) Light Forcing Hierarchical Sparse
+ * Attention (HSA) library, liblf_hsa.so.
+ *
+ * One HSA attention call of a chunked autoregressive video diffusion
+ * transformer, as described in "Light Forcing：通过稀疏注意力加速自回归视频扩散"
+ * (paper.rainbus.top, execution-flow paragraph, stages 2 and 3) and
+ * "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
+ * Attention" (gist.science, Technical Summary 2.2):
+ *
+ *   lf_pool              block mean pooling of q and k, frame mean pooling of k
+ *   lf_select_frames     per query block: frame scores, top-k memory frames T_r
+ *                        plus the always-kept sink / recent / current frames
+ *   lf_select_blocks     per selected frame: block scores, top-k blocks J_r(tau),
+ *                        written as a compacted block list (the mask B_r)
+ *   lf_block_sparse_attn softmax attention of each query block over the valid
+ *                        tokens of its listed KV blocks (tcgen05 tensor cores)
+ *
+ * plus the host-side Chunk-Aware Growth budget solver (same pages, stage 1 /
+ * Technical Summary 2.1).
+ *
+ * Conventions shared by every device entry point
+ * ----------------------------------------------
+ * - Layout: q and out are [batch, heads, n_cur*frame_tokens, head_dim] bf16,
+ *   contiguous. k and v are [batch, heads, kv_stride, head_dim] bf16: head
+ *   (b,h) starts at token (b*heads + h) * kv_stride and its first
+ *   n_frames*frame_tokens tokens are the call's KV frames, in the order
+ *   [sink frames][memory frames][recent frames][current-chunk frames].
+ *   Queries are the current-chunk frames.
+ * - Blocks are block_tokens = 64 consecutive tokens of one frame; a frame of F
+ *   tokens has bpf = ceil(F/64) blocks and its last block may be partial (it
+ *   holds F - 64*(bpf-1) tokens). Query block r = f*bpf + j is block j of
+ *   current-chunk frame f (Rq = n_cur*bpf blocks); KV block g = tau*bpf + j is
+ *   block j of KV frame tau (Nkv = n_frames*bpf blocks).
+ * - bf16 data is passed as uint16_t bit patterns; pooled data is fp32.
+ * - Ownership: the caller allocates every device buffer (inputs, outputs and
+ *   the intermediate pooled / selection buffers). The library never allocates,
+ *   frees or synchronises; each call only enqueues kernels on `stream`
+ *   (a cudaStream_t; NULL = the legacy default stream) and returns.
+ * - Device pointers must be 16-byte aligned (the attention kernel reads them
+ *   with TMA). Arguments are validated before anything is launched; a failed
+ *   validation launches nothing.
+ * - Device-side faults that only the kernel can see (an out-of-range block id
+ *   in a list, a bounded wait that expired) never trap: the kernel records a
+ *   code in a per-device error word and returns; lf_get_device_error() reads
+ *   and clears it.
+ */
+#ifndef LF_HSA_H
+#define LF_HSA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LF_API __attribute__((visibility("default")))
+#else
+#define LF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lf_status {
+    LF_OK = 0,
+    LF_ERR_NULL = 1,           /* a required pointer is NULL */
+    LF_ERR_ALIGN = 2,          /* a device pointer is not 16-byte aligned */
+    LF_ERR_SHAPE = 3,          /* sizes outside the supported set (see lf_hsa_shape) */
+    LF_ERR_TOPK = 4,           /* a top-k count below 1 */
+    LF_ERR_CAP = 5,            /* list_cap smaller than the list the call writes */
+    LF_ERR_INFEASIBLE = 6,     /* CAG: beta < 0 or some s_i outside [0, 1) */
+    LF_ERR_CUDA = 7,           /* a CUDA runtime / launch call failed */
+    LF_ERR_DEVICE_TIMEOUT = 8, /* device error word: a bounded wait in a kernel expired */
+    LF_ERR_ARG = 9,            /* another invalid scalar (chunk index, sparsity, scale) */
+    LF_ERR_LIST = 10,          /* device error word: a block id or count out of range */
+    LF_ERR_NO_DEVICE = 11      /* no usable sm_100 device */
+} lf_status;
+
+/*
+ * Sizes of one HSA call.
+ *   batch, heads >= 1; head_dim in {64, 128}; block_tokens == 64;
+ *   1 <= frame_tokens <= 8192 (so bpf <= 128);
+ *   n_sink, n_recent >= 0, n_cur >= 1, n_sink + n_recent + n_cur <= n_frames;
+ *   the number of memory frames n_frames - n_sink - n_recent - n_cur <= 1024;
+ *   kv_stride = 0 means n_frames*frame_tokens, otherwise >= that.
+ */
+typedef struct lf_hsa_shape {
+    int32_t batch;
+    int32_t heads;
+    int32_t head_dim;
+    int32_t frame_tokens;
+    int32_t block_tokens;
+    int32_t n_frames;
+    int32_t n_sink;
+    int32_t n_recent;
+    int32_t n_cur;
+    int64_t kv_stride;
+} lf_hsa_shape;
+
+/*
+ * Token compression (paper.rainbus.top, execution flow, stage 2; gist.science
+ * Technical Summary 2.2 "Token Compression").
+ *   q_pool  [B,H,Rq,D]  fp32: mean of the tokens of each query block
+ *   k_pool  [B,H,Nkv,D] fp32: mean of the tokens of each KV block
+ *   k_frame [B,H,NF,D]  fp32: mean of all tokens of each KV frame (k^ of the
+ *                              memory frames is the slice [n_sink, n_sink+n_mem))
+ * Partial blocks are averaged over their real tokens. Reads q and k once.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_pool(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                  float* q_pool, float* k_pool, float* k_frame, void* stream);
+
+/* Number of frames in each T_r: n_frames when chunk_index == 1, else
+ * n_sink + min(topk_frames, n_mem) + n_recent + n_cur. Returns -1 on a bad shape. */
+LF_API int32_t lf_frames_selected(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames);
+
+/*
+ * Frame-level selection (paper.rainbus.top, execution flow, stage 3, first
+ * level: p_r = <q~_r, k^_M>, top-k frames T_r, sink / most recent / current
+ * chunk frames always kept; gist.science Technical Summary 2.2 "Frame
+ * Selection").
+ *   chunk_index  1-based position of the chunk in the rollout; chunk 1 is
+ *                dense (stage 1) and selects every frame.
+ *   topk_frames  k_f >= 1; values above n_mem keep every memory frame.
+ *   frame_sel    [B,H,Rq,n_sel] int32 out, n_sel = lf_frames_selected(...):
+ *                the frame ids of T_r in ascending order.
+ * Scores are fp32 inner products; among equal scores the lower frame id wins.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_TOPK, LF_ERR_ARG,
+ * LF_ERR_CUDA.
+ */
+LF_API lf_status lf_select_frames(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames,
+                           const float* q_pool, const float* k_frame, int32_t* frame_sel,
+                           void* stream);
+
+/* Length of each block list row: n_sel * min(topk_blocks, bpf) (n_frames*bpf
+ * for chunk 1). Returns -1 on a bad shape. */
+LF_API int32_t lf_list_capacity(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames,
+                         int32_t topk_blocks);
+
+/*
+ * Block-level selection (paper.rainbus.top, execution flow, stage 3, second
+ * level: o_r(tau,j) = <q~_r, k~_j^(tau)>, top-k blocks J_r(tau) inside each
+ * selected frame, mask B_r(tau,j) = 1[tau in T_r, j in J_r(tau)];
+ * gist.science Technical Summary 2.2 "Block Selection").
+ *   frame_sel    [B,H,Rq,n_sel] int32 from lf_select_frames (same chunk_index
+ *                and topk_frames).
+ *   topk_blocks  k_b >= 1; values above bpf keep every block of a frame.
+ *   block_list   [B,H,Rq,list_cap] int32 out: row (b,h,r) holds the global KV
+ *                block ids tau*bpf + j of the mask, frame by frame in the order
+ *                of frame_sel and ascending j inside a frame (so the row is
+ *                ascending when frame_sel is). Entries past the count are not
+ *                written.
+ *   block_count  [B,H,Rq] int32 out: n_sel * min(topk_blocks, bpf) per row
+ *                (every row keeps the same number of blocks).
+ *   list_cap     >= lf_list_capacity(...), else LF_ERR_CAP.
+ * Among equal scores the lower block index wins.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_TOPK, LF_ERR_CAP,
+ * LF_ERR_ARG, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames,
+                           int32_t topk_blocks, const float* q_pool, const float* k_pool,
+                           const int32_t* frame_sel, int32_t* block_list, int32_t* block_count,
+                           int32_t list_cap, void* stream);
+
+/*
+ * Block-sparse softmax attention (paper.rainbus.top, execution flow, stage 3,
+ * final step: attention over the block mask).
+ *   out[b,h,t,:] = sum_s softmax_s(scale * <q_t, k_s>) v_s over every valid
+ *   token s of the KV blocks listed for t's query block (no causal mask).
+ *   block_list / block_count as written by lf_select_blocks (any order, no
+ *   duplicates expected); list_cap is the row stride of block_list.
+ *   softmax_scale <= 0 selects 1/sqrt(head_dim).
+ *   out [B,H,Lq,D] bf16: every valid query row is written; a row whose list is
+ *   empty gets zeros.
+ * Block ids outside [0, Nkv) or counts outside [0, list_cap] are skipped /
+ * clamped on the device and reported as LF_ERR_LIST by lf_get_device_error().
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_CAP, LF_ERR_ARG,
+ * LF_ERR_NO_DEVICE, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const int32_t* block_list,
+                               const int32_t* block_count, int32_t list_cap, float softmax_scale,
+                               uint16_t* out, void* stream);
+
+/*
+ * Chunk-Aware Growth budget solver, host only, fp64 (paper.rainbus.top,
+ * execution flow, stage 1; gist.science Technical Summary 2.1; 163.com
+ * article section 2).
+ *   s_1 = 0 (first chunk dense); s_i = s_base - alpha_i * beta for i > 1 with
+ *   alpha_i = 1/sqrt(T[i-1]); beta solves
+ *       sum_i w_i s_i = s_target * sum_i w_i
+ *   over all chunks (target_over_all != 0) or over chunks 2..n (== 0).
+ *   flops_w = NULL uses w_i = i (dense attention FLOPs of chunk i when the KV
+ *   length grows by one chunk per step).
+ *   s_out[n_chunks] and *beta_out are written whenever the arguments are valid,
+ *   also when the result is infeasible.
+ * Errors: LF_ERR_NULL, LF_ERR_ARG (n_chunks < 2, a T or w <= 0, s outside
+ * [0,1)), LF_ERR_INFEASIBLE (beta < 0 or some s_i outside [0,1)).
+ */
+LF_API lf_status lf_cag_budget(int32_t n_chunks, const double* T, const double* flops_w, double s_base,
+                        double s_target, int32_t target_over_all, double* s_out,
+                        double* beta_out);
+
+/*
+ * Per-frame block count for a target block sparsity s in [0,1): the kept
+ * (1 - s) * n_kv_blocks blocks spread evenly over n_sel selected frames,
+ * rounded to nearest and clamped to [1, bpf]. The pages give no formula for
+ * this step; this is the plainest reading. Returns -1 on invalid arguments.
+ */
+LF_API int32_t lf_blocks_for_sparsity(double s, int32_t n_kv_blocks, int32_t n_sel_frames, int32_t bpf);
+
+/* Reads and clears the error word of the current device: LF_OK or
+ * LF_ERR_DEVICE_TIMEOUT / LF_ERR_LIST. Synchronises the current device. */
+LF_API lf_status lf_get_device_error(int32_t* detail);
+
+/* Static description of a status code. */
+LF_API const char* lf_status_string(lf_status status);
+
+/* Library version, e.g. "lf_hsa 0.1.0 sm_100a". */
+LF_API const char* lf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LF_HSA_H */

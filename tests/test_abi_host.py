@@ -1,0 +1,156 @@
+"""The C-ABI library loads, exports what include/lf_hsa.h declares, and its host
+logic (CAG solver, block-count mapping, sizes, argument validation) matches the
+oracle. No CUDA device is touched: every device entry point called here fails
+validation before it could launch anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_lf_b200 as L
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lf_hsa.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^LF_API\s+[\w\s\*]+?\b(lf_\w+)\(", txt, re.M)))
+
+
+def test_exports_match_header():
+    declared = _declared()
+    assert declared == sorted(L.ABI_FUNCTIONS)
+    out = os.popen(f"nm -D --defined-only {L.LIB_PATH}").read()
+    exported = sorted(m.group(1) for m in re.finditer(r" T (lf_\w+)$", out, re.M))
+    assert exported == declared
+    for name in declared:
+        assert hasattr(L.lib, name)
+
+
+def test_shape_struct_layout():
+    # 9 int32 fields, 4 bytes of padding, one int64
+    assert ctypes.sizeof(L.LfShape) == 48
+    assert L.LfShape.kv_stride.offset == 40
+
+
+def test_version():
+    assert "sm_100a" in L.lf_version()
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_cag_matches_oracle(seed):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(2, 10))
+    T = np.cumsum(rng.uniform(0.2, 3.0, n))
+    w = rng.uniform(0.1, 4.0, n) if seed % 3 else None
+    s_base = rng.uniform(0.6, 0.99)
+    s_target = rng.uniform(0.05, 0.95) * s_base
+    over_all = bool(seed % 2)
+    st, s, beta = L.lf_cag_budget(list(T), None if w is None else list(w), s_base, s_target, over_all)
+    rc, so, bo = oracle.cag(T, w, s_base, s_target, over_all)
+    assert (st == 0) == (rc == 0)
+    if st in (0, 6):  # values are reported for feasible and infeasible budgets
+        assert beta == pytest.approx(bo, rel=1e-12, abs=1e-15)
+        np.testing.assert_allclose(s, so, rtol=1e-12, atol=1e-15)
+
+
+def test_cag_errors():
+    assert L.lf_cag_budget([1.0], None, 0.9, 0.5)[0] == 9                 # one chunk
+    assert L.lf_cag_budget([1.0, 0.0], None, 0.9, 0.5)[0] == 9            # T <= 0
+    assert L.lf_cag_budget([1.0, 2.0], [1.0, -1.0], 0.9, 0.5)[0] == 9     # w <= 0
+    assert L.lf_cag_budget([1.0, 2.0], None, 1.2, 0.5)[0] == 9            # s_base outside [0,1)
+    assert L.lf_cag_budget([1.0, 2.0, 3.0], None, 0.5, 0.6)[0] == 6       # beta < 0
+    assert L.lib.lf_cag_budget(3, None, None, 0.9, 0.5, 1, None, None) == 1
+
+
+def test_cag_rollout_default_matches_oracle():
+    st, s, beta = L.lf_cag_budget(list(range(1, 8)), None, 0.95, 0.80, True)
+    rc, so, bo = oracle.cag(np.arange(1, 8), np.arange(1, 8), 0.95, 0.80, True)
+    assert st == 0 and rc == 0
+    assert beta == pytest.approx(bo, rel=1e-14)
+    np.testing.assert_allclose(s, so, rtol=1e-14)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.3, 0.5, 0.79, 0.8, 0.81, 0.9, 0.95, 0.999])
+@pytest.mark.parametrize("nkv,nsel,bpf", [(525, 9, 25), (1625, 9, 25), (36, 6, 4), (75, 6, 25)])
+def test_blocks_for_sparsity_matches_oracle(s, nkv, nsel, bpf):
+    assert L.lf_blocks_for_sparsity(s, nkv, nsel, bpf) == oracle.blocks_for_sparsity(s, nkv, nsel, bpf)
+
+
+def test_sizes_match_oracle():
+    for (NF, ns, nr, nc) in [(21, 1, 1, 3), (9, 1, 1, 2), (3, 0, 0, 3), (65, 1, 1, 3), (5, 2, 0, 3)]:
+        sh = L.LfShape.make(1, 2, 128, 1560, NF, ns, nr, nc)
+        os_ = oracle.Shape(1, 2, 128, 1560, 64, NF, ns, nr, nc)
+        for chunk in (1, 2, 5):
+            for kf in (1, 4, 100):
+                n = L.lf_frames_selected(sh, chunk, kf)
+                assert n == oracle.frames_selected(os_, chunk, kf)
+                for kb in (1, 12, 25, 40):
+                    per = 25 if chunk == 1 else min(kb, 25)
+                    assert L.lf_list_capacity(sh, chunk, kf, kb) == n * per
+
+
+def _shape(**kw):
+    base = dict(batch=1, heads=2, head_dim=128, frame_tokens=1560, n_frames=21, n_sink=1,
+                n_recent=1, n_cur=3)
+    base.update(kw)
+    return L.LfShape.make(**base)
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(head_dim=96), 3), (dict(block_tokens=32), 3), (dict(frame_tokens=0), 3),
+    (dict(frame_tokens=9000), 3), (dict(n_cur=0), 3), (dict(n_frames=4), 3),
+    (dict(n_sink=-1), 3), (dict(batch=0), 3), (dict(kv_stride=100), 3),
+    (dict(n_frames=1030, n_sink=1, n_recent=1, n_cur=3), 3),
+])
+def test_shape_validation(bad, code):
+    sh = _shape(**bad)
+    p = ctypes.c_void_p(FAKE)
+    assert L.lib.lf_pool(ctypes.byref(sh), p, p, p, p, p, None) == code
+    assert L.lib.lf_select_frames(ctypes.byref(sh), 2, 4, p, p, p, None) == code
+    assert L.lib.lf_select_blocks(ctypes.byref(sh), 2, 4, 12, p, p, p, p, p, 1000, None) == code
+    assert L.lib.lf_block_sparse_attn(ctypes.byref(sh), p, p, p, p, p, 1000, 0.0, p, None) == code
+    assert L.lf_frames_selected(sh, 2, 4) == -1
+    assert L.lf_list_capacity(sh, 2, 4, 12) == -1
+
+
+def test_argument_validation():
+    sh = _shape()
+    p = ctypes.c_void_p(FAKE)
+    mis = ctypes.c_void_p(FAKE + 8)
+    S = ctypes.byref(sh)
+    assert L.lib.lf_pool(None, p, p, p, p, p, None) == 1
+    assert L.lib.lf_pool(S, None, p, p, p, p, None) == 1
+    assert L.lib.lf_pool(S, p, mis, p, p, p, None) == 2
+    assert L.lib.lf_select_frames(S, 0, 4, p, p, p, None) == 9      # chunk index is 1-based
+    assert L.lib.lf_select_frames(S, 2, 0, p, p, p, None) == 4      # top-k below 1
+    assert L.lib.lf_select_frames(S, 2, 4, p, None, p, None) == 1
+    assert L.lib.lf_select_frames(S, 2, 4, p, p, mis, None) == 2
+    assert L.lib.lf_select_blocks(S, 2, 4, 0, p, p, p, p, p, 108, None) == 4
+    assert L.lib.lf_select_blocks(S, 2, 4, 12, p, p, p, p, p, 107, None) == 5   # cap < 9*12
+    assert L.lib.lf_select_blocks(S, 2, 4, 12, p, p, p, None, p, 108, None) == 1
+    assert L.lib.lf_block_sparse_attn(S, p, p, p, p, p, -1, 0.0, p, None) == 5
+    assert L.lib.lf_block_sparse_attn(S, p, p, p, p, p, 108, float("nan"), p, None) == 9
+    assert L.lib.lf_block_sparse_attn(S, p, p, None, p, p, 108, 0.0, p, None) == 1
+    assert L.lib.lf_block_sparse_attn(S, p, p, p, p, p, 108, 0.0, mis, None) == 2
+
+
+def test_status_strings():
+    for code in range(12):
+        assert L.lf_status_string(code)
+    assert L.lf_status_string(99) == "unknown status"
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    sh = _shape(heads=1, n_frames=5, n_sink=1, n_recent=1, n_cur=1, frame_tokens=64)
+    q = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.lf_pool(sh, q, q, q.float(), q.float(), q.float())

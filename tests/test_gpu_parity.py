@@ -1,0 +1,116 @@
+"""GPU parity of the whole HSA call against the fp64 oracle, through the C ABI.
+
+Small cases are checked element by element (every pooled value, every mask row
+under the tie rule, every output row); they span several tiles, ragged frames
+(partial 64-token blocks), odd list lengths, frames shorter than one block, a
+KV head stride larger than the used length, the dense first chunk, all-keep
+masks and sharp softmaxes that force many online-softmax rescales. The five
+named workloads run at full size in the launch configuration the benchmark
+uses, with every mask row and pooled value checked and a sample of output rows
+recomputed by the oracle.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import lf_synth
+import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand(seed, B, H, Lq, Lkv, D, kscale=1.0, kv_stride=0):
+    g = torch.Generator().manual_seed(seed)
+    Ls = kv_stride or Lkv
+    q = torch.randn(B, H, Lq, D, generator=g).to(torch.bfloat16)
+    k = (torch.randn(B, H, Ls, D, generator=g) * kscale).to(torch.bfloat16)
+    v = torch.randn(B, H, Ls, D, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def _full_check(shape, q, k, v, chunk, kf, kb, kv_stride=0, rows=None):
+    g = parity.run_gpu(shape, q, k, v, chunk, kf, kb, kv_stride=kv_stride)
+    s_or = oracle.Shape(shape.batch, shape.heads, shape.head_dim, shape.frame_tokens, 64,
+                        shape.n_frames, shape.n_sink, shape.n_recent, shape.n_cur, kv_stride=kv_stride)
+    qp, kp, kfr = oracle.pool(s_or, q, k)
+    sel, fsc = oracle.select_frames(s_or, chunk, kf, qp, kfr)
+    o = dict(q_pool=qp, k_pool=kp, k_frame=kfr, frame_sel=sel, frame_scores=fsc)
+    parity.check_pool(g, o, q, k)
+    fr = parity.check_frames(s_or, chunk, kf, g, o)
+    bl = parity.check_blocks(s_or, chunk, kb, g, qp, kp)
+    at = parity.check_attention(s_or, q, k, v, g, rows=rows)
+    return fr, bl, at
+
+
+SMALL = [
+    # name, B, H, D, F, (n_sink, n_mem, n_recent, n_cur), chunk, kf, kb, kscale, kv_pad
+    ("ragged_d128", 2, 3, 128, 200, (1, 2, 1, 3), 2, 1, 2, 1.0, 0),
+    ("ragged_d64_odd_lists", 1, 2, 64, 100, (1, 2, 1, 1), 2, 2, 1, 1.0, 0),
+    ("frame_shorter_than_block", 1, 2, 128, 40, (1, 3, 1, 2), 2, 2, 1, 1.0, 0),
+    ("exact_blocks", 2, 2, 128, 128, (1, 4, 1, 2), 2, 2, 1, 1.0, 0),
+    ("kv_head_stride", 2, 2, 128, 150, (1, 3, 1, 2), 2, 2, 2, 1.0, 77),
+    ("dense_first_chunk", 1, 2, 128, 260, (0, 0, 0, 3), 1, 4, 2, 1.0, 0),
+    ("all_keep", 1, 2, 128, 190, (1, 2, 1, 2), 2, 9, 9, 1.0, 0),
+    ("no_memory_frames", 1, 2, 128, 130, (1, 0, 1, 2), 2, 4, 2, 1.0, 0),
+    ("no_sink_no_recent", 1, 2, 64, 256, (0, 5, 0, 2), 2, 2, 3, 1.0, 0),
+    ("sharp_softmax_rescales", 1, 2, 128, 300, (1, 4, 1, 2), 2, 3, 3, 8.0, 0),
+    ("long_lists_many_tiles", 1, 2, 128, 1560, (1, 7, 1, 1), 2, 7, 25, 1.0, 0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_cases_full(case):
+    name, B, H, D, F, (ns, nm, nr, nc), chunk, kf, kb, kscale, pad = case
+    NF = ns + nm + nr + nc
+    shape = oracle.Shape(B, H, D, F, 64, NF, ns, nr, nc)
+    stride = NF * F + pad if pad else 0
+    q, k, v = _rand(zlib.crc32(name.encode()) % 1000, B, H, nc * F, NF * F, D, kscale, stride)
+    _full_check(shape, q, k, v, chunk, kf, kb, kv_stride=stride)
+
+
+def test_tiny_workload_full():
+    w = lf_synth.CONFIGS["tiny"]
+    q, k, v = lf_synth.make_qkv(w)
+    shape = oracle.shape_of(w)
+    fr, bl, at = _full_check(shape, q, k, v, w.chunk_index, w.topk_frames, w.topk_blocks)
+    assert fr["exact"] > 0
+
+
+def _kb(w, shape):
+    if w.topk_blocks:
+        return w.topk_blocks
+    n_sel = oracle.frames_selected(shape, w.chunk_index, w.topk_frames)
+    return oracle.blocks_for_sparsity(w.sparsity, shape.Nkv, n_sel, shape.bpf)
+
+
+@pytest.mark.parametrize("name,kb_override", [("layer480p", None), ("longvideo480p", None),
+                                              ("patterns480p", None), ("patterns480p", 6)])
+def test_full_size_workloads(name, kb_override):
+    w = lf_synth.CONFIGS[name]
+    q, k, v = lf_synth.make_qkv(w)
+    shape = oracle.shape_of(w)
+    kb = kb_override or _kb(w, shape)
+    rows = parity.sample_rows(shape, per_block=3, blocks_per_head=5, seed=1)
+    fr, bl, at = _full_check(shape, q, k, v, w.chunk_index, w.topk_frames, kb, rows=rows)
+    # the planted structure makes most frame cuts clear
+    assert fr["exact"] >= 0.5 * (fr["exact"] + fr["tie"])
+
+
+def test_rollout_chunks():
+    """The 7-chunk rollout: chunk 1 dense, chunks 2-7 with the Chunk-Aware Growth budgets."""
+    w = lf_synth.CONFIGS["rollout480p"]
+    qa, ka, va = lf_synth.make_rollout_qkv(w)
+    n_chunks = int(w.extra["n_chunks"])
+    rc, s, beta = oracle.cag(np.arange(1, n_chunks + 1), np.arange(1, n_chunks + 1),
+                             w.extra["s_base"], w.sparsity, True)
+    assert rc == 0
+    for chunk in range(1, n_chunks + 1):
+        wc, q, k, v = lf_synth.rollout_chunk(w, qa, ka, va, chunk)
+        shape = oracle.shape_of(wc)
+        n_sel = oracle.frames_selected(shape, chunk, w.topk_frames)
+        kb = shape.bpf if chunk == 1 else oracle.blocks_for_sparsity(s[chunk - 1], shape.Nkv, n_sel, shape.bpf)
+        rows = parity.sample_rows(shape, per_block=2, blocks_per_head=3, seed=chunk)
+        _full_check(shape, q, k, v, chunk, w.topk_frames, kb, rows=rows)
