@@ -126,6 +126,23 @@ bool encode_rows(CUtensorMap* m, const void* base, long long rows, int D, int bo
     return r == CUDA_SUCCESS;
 }
 
+// 4-D bf16 view of a [rows, 128] tensor as {64 elems, 8 rows, 2 panels,
+// rows/8 groups} with a {64, 8, 2, groups} box: one box brings a block of
+// 8*groups rows in the interleaved [group][panel][8 rows x 128 B] layout.
+bool encode_blocks_il(CUtensorMap* m, const void* base, long long rows, int groups)
+{
+    auto fn = encode_fn();
+    if (!fn || rows % 8 != 0) return false;
+    const cuuint64_t dims[4] = {64u, 8u, 2u, static_cast<cuuint64_t>(rows / 8)};
+    const cuuint64_t strides[3] = {256u, 128u, 2048u};
+    const cuuint32_t box[4] = {64u, 8u, 2u, static_cast<cuuint32_t>(groups)};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -241,13 +258,19 @@ lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t* q, con
     const long long BH = static_cast<long long>(d.B) * d.H;
     lf::AttnMaps m;
     const long long q_rows = BH * d.Lq, kv_rows = BH * d.kv_stride;
-    if (!encode_rows(&m.q, q, q_rows, d.D, 64) || !encode_rows(&m.q_rem, q, q_rows, d.D, d.rem) ||
-        !encode_rows(&m.k, k, kv_rows, d.D, 64) || !encode_rows(&m.k_rem, k, kv_rows, d.D, d.rem) ||
-        !encode_rows(&m.v, v, kv_rows, d.D, 64) || !encode_rows(&m.v_rem, v, kv_rows, d.D, d.rem))
+    if (!encode_rows(&m.q, q, q_rows, d.D, 64) || !encode_rows(&m.q_rem, q, q_rows, d.D, d.rem)) return LF_ERR_CUDA;
+    // One box per KV block when every block starts on an 8-row boundary.
+    bool interleaved = d.D == 128 && d.F % 8 == 0 && d.kv_stride % 8 == 0 &&
+                       encode_blocks_il(&m.k, k, kv_rows, 8) && encode_blocks_il(&m.k_rem, k, kv_rows, d.rem / 8) &&
+                       encode_blocks_il(&m.v, v, kv_rows, 8) && encode_blocks_il(&m.v_rem, v, kv_rows, d.rem / 8);
+    if (!interleaved &&
+        (!encode_rows(&m.k, k, kv_rows, d.D, 64) || !encode_rows(&m.k_rem, k, kv_rows, d.D, d.rem) ||
+         !encode_rows(&m.v, v, kv_rows, d.D, 64) || !encode_rows(&m.v_rem, v, kv_rows, d.D, d.rem)))
         return LF_ERR_CUDA;
     lf::AttnArgs a{block_list, block_count, out, list_cap, d.Rq, d.bpf, d.F, d.Lq, d.Nkv, d.rem, d.kv_stride,
                    scale * 1.4426950408889634f, err};
-    return launch_status(lf::launch_attn(m, a, d.D, static_cast<int>(BH * d.Rq), static_cast<cudaStream_t>(stream)));
+    return launch_status(
+        lf::launch_attn(m, a, d.D, interleaved, static_cast<int>(BH * d.Rq), static_cast<cudaStream_t>(stream)));
 }
 
 lf_status lf_cag_budget(int32_t n_chunks, const double* T, const double* flops_w, double s_base, double s_target,

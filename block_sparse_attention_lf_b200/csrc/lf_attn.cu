@@ -10,28 +10,41 @@
 //   * KV-major formulation. A tile is two listed KV blocks (128 tokens). The
 //     tensor core computes S^T = K_tile * Q^T (M = 128 KV tokens, N = 64
 //     queries, K = head_dim) into TMEM, and O^T += V_tile^T * P^T (M = 128
-//     head-dim rows, N = 64 queries, K = 128 KV tokens). Both MMAs therefore
-//     run with M = 128 on exactly the listed blocks, with no union of
-//     neighbouring query blocks' lists.
-//   * Warp roles (320 threads): warp 0 issues TMA loads (Q once; per tile the
-//     listed K and V blocks, 64-row boxes, 128-byte swizzle), warp 1 allocates
-//     TMEM and issues tcgen05.mma from one thread, warps 2-9 are two softmax
-//     warpgroups. TMEM lane t of S^T is KV token t of the tile, so each
-//     softmax thread owns one KV token and 32 query columns (warpgroup 0:
-//     queries 0-31, warpgroup 1: queries 32-63).
+//     head-dim rows, N = 64 queries, K = 128 KV tokens). Both MMAs run with
+//     M = 128 (M = 64 issues at half rate on this part) on exactly the listed
+//     blocks, with no union of neighbouring query blocks' lists.
+//   * Gather. K and V dominate the traffic (each query block reads its own
+//     ~100 blocks from L2). Small TMA boxes cap the per-SM L2 bandwidth, so
+//     for head_dim 128 each 64-token block (16 KB, contiguous) arrives as ONE
+//     4-D box {64 elems, 8 rows, 2 panels, 8 row groups} that lands in an
+//     interleaved layout [row group][panel][8 rows x 128 B] (128-byte swizzle).
+//     Its 8-row groups sit a uniform 2 KB apart, so one smem descriptor spans
+//     both blocks of a tile for the S^T MMA (SBO = 2 KB, panel at +1 KB) and
+//     for the PV MMA (MN-major: LBO = 1 KB between head-dim panels, SBO = 2 KB
+//     between 8-row groups). Frames whose token count is not a multiple of 8,
+//     and head_dim 64, use 2-D boxes per 64-wide panel into a plain
+//     [panel][row] layout instead.
+//   * Warp roles (384 threads): warp 0 issues the Q and K loads, warp 1 the V
+//     loads (so a V slot that is still in use never delays K prefetch), warp 2
+//     allocates TMEM and issues tcgen05.mma from one thread, warp 3 idles,
+//     warps 4-11 are two softmax warpgroups. TMEM lane t of S^T is KV token t
+//     of the tile, so each softmax thread owns one KV token and 32 query
+//     columns (warpgroup 0: queries 0-31, warpgroup 1: queries 32-63).
 //   * Online softmax in fp32, base 2, with a lazy stabiliser: each query
-//     column keeps m (running max of scale*log2(e)*score); a tile whose scores
-//     stay within m + 8 (p <= 256) is exponentiated against the current m with
-//     no cross-thread work; only when some score exceeds that bound does the
-//     warpgroup compute the exact column maxima of the tile (butterfly
-//     reductions + shared memory) and rescale its columns of O^T in TMEM. Row
-//     sums are kept per thread and reduced once at the end.
+//     column keeps m (running max of scale*log2(e)*score, in shared memory); a
+//     tile whose scores stay within m + 8 (p <= 256) is exponentiated against
+//     the current m with no cross-thread work; only when some score exceeds
+//     that bound does the warpgroup compute the exact column maxima of the tile
+//     (butterfly reductions + shared memory) and rescale its columns of O^T in
+//     TMEM. Row sums are kept per thread and reduced once at the end.
 //   * P^T goes to shared memory as bf16 in the 128-byte-swizzled MN-major
 //     layout the MMA reads; masked KV tokens (past the end of a partial block,
 //     or the unused half of an odd last tile) get P = 0.
-//   * Pipelines: K ring of 2 slots, V ring of 3, S double-buffered in TMEM, P
-//     double-buffered in shared memory; the MMA thread issues S for tile i+2
-//     right after PV for tile i, so S is ready before the softmax needs it.
+//   * Pipelines: K ring of 3 slots, V ring of 2, S double-buffered in TMEM, P
+//     double-buffered in shared memory. The softmax releases an S buffer as
+//     soon as the scores are in registers, and the MMA thread then issues S
+//     for tile i+2 before PV for tile i, so the tensor pipe works on the next
+//     scores while the softmax exponentiates.
 //   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
@@ -41,46 +54,62 @@
 
 #include <cuda_bf16.h>
 
+#include <cstddef>
+
 namespace lf {
 namespace {
 
-constexpr int ATTN_THREADS = 320;
-constexpr int KSLOTS = 2;
-constexpr int VSLOTS = 3;
+constexpr int ATTN_THREADS = 384;
+constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_SOFT0 = 4;
+constexpr int KSLOTS = 3;
+constexpr int VSLOTS = 2;
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
 constexpr uint32_t TMEM_COLS = 256;         // S0: 0-63, S1: 64-127, O^T: 128-191
+constexpr int ROWS_SMEM = 1024;             // list entries whose row counts are cached in smem
 
-template <int D>
+// Shared-memory plan. IL selects the interleaved K/V layout (head_dim 128,
+// one 4-D box per block); otherwise K/V use [panel][128 rows x 128 B].
+template <int D, bool IL>
 struct AttnLayout {
-    static constexpr int NP = D / 64;                       // 64-element panels of head_dim
-    static constexpr uint32_t PANEL_Q = 64u * 128u;          // 64 rows x 128 B
-    static constexpr uint32_t PANEL_KV = 128u * 128u;        // 128 rows x 128 B
+    static constexpr int NP = D / 64;                  // 64-element panels of head_dim
+    static constexpr uint32_t PANEL_Q = 64u * 128u;     // 64 rows x 128 B
+    static constexpr uint32_t PANEL_KV = 128u * 128u;   // 128 rows x 128 B (panel layout)
+    static constexpr uint32_t BLOCK_IL = 16384u;        // one 64 x 128 bf16 block (interleaved)
     static constexpr uint32_t Q_BYTES = NP * PANEL_Q;
     static constexpr uint32_t K_SLOT = NP * PANEL_KV;
-    static constexpr uint32_t V_SLOT = 2u * PANEL_KV;        // always 2 panels: the PV MMA has M = 128
-    static constexpr uint32_t P_BUF = 128u * 128u;           // P^T: 128 KV rows x 64 queries bf16
+    static constexpr uint32_t V_SLOT = 2u * PANEL_KV;   // the PV MMA has M = 128 head-dim rows
+    static constexpr uint32_t P_BUF = 128u * 128u;      // P^T: 128 KV rows x 64 queries bf16
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + KSLOTS * K_SLOT;
     static constexpr uint32_t OFF_P = OFF_V + VSLOTS * V_SLOT;
     static constexpr uint32_t OFF_AUX = OFF_P + 2u * P_BUF;
+    // smem descriptor strides of the K/V tiles
+    static constexpr uint32_t KV_SBO = IL ? 2048u : 1024u;          // between 8-row groups
+    static constexpr uint32_t KV_PANEL = IL ? 1024u : PANEL_KV;     // between 64-wide panels
+    static constexpr uint32_t KV_K16 = IL ? 4096u : 2048u;          // 16 KV rows (one PV k-step)
+    static_assert(!IL || D == 128, "interleaved layout is for head_dim 128");
 };
 
 struct AttnAux {
     uint64_t q_full;
     uint64_t k_full[KSLOTS], k_empty[KSLOTS];
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
-    uint64_t s_full[2], p_full[2], p_empty[2];
+    uint64_t s_full[2], s_free[2], p_full[2], p_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
     float red[2][4][32];
+    alignas(16) float m_s[2][32];  // running max (log2 units) of each query column (read as float4)
+    uint8_t rows[ROWS_SMEM];       // valid token rows of list entry b (0: not a valid block)
 };
 
-template <int D>
+static_assert(offsetof(AttnAux, m_s) % 16 == 0, "m_s is read with 16-byte loads");
+
+template <int D, bool IL>
 constexpr uint32_t attn_smem_bytes()
 {
-    return AttnLayout<D>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux)) + 1024u;
+    return AttnLayout<D, IL>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux)) + 1024u;
 }
 
 template <bool MAX>
@@ -110,14 +139,40 @@ __device__ __forceinline__ int block_rows(const AttnArgs& a, int g, int bh, int*
     return (j == a.bpf - 1) ? a.rem : 64;
 }
 
-template <int D>
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Load one KV block (`rows` valid tokens starting at flattened row `first`)
+// into half `h` of a K or V slot.
+template <int D, bool IL>
+__device__ __forceinline__ void load_block(uint8_t* slot, int h, int rows, int first, const CUtensorMap* full,
+                                           const CUtensorMap* part, uint64_t* bar)
+{
+    using L = AttnLayout<D, IL>;
+    const CUtensorMap* m = rows == 64 ? full : part;
+    if constexpr (IL) {
+        tma_load_4d(slot + h * L::BLOCK_IL, m, 0, 0, 0, first >> 3, bar);
+    } else {
+#pragma unroll
+        for (int p = 0; p < L::NP; ++p) tma_load_2d(slot + p * L::PANEL_KV + h * 64 * 128, m, p * 64, first, bar);
+    }
+}
+
+template <int D, bool IL>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rem,
             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k_rem,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_v_rem,
             const AttnArgs a)
 {
-    using L = AttnLayout<D>;
+    using L = AttnLayout<D, IL>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     AttnAux& x = *reinterpret_cast<AttnAux*>(smem + L::OFF_AUX);
@@ -144,16 +199,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int s = 0; s < VSLOTS; ++s) { mbar_init(&x.v_full[s], 1); mbar_init(&x.v_empty[s], 1); }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&x.s_full[s], 1);
-            mbar_init(&x.p_full[s], 256);
+            mbar_init(&x.s_free[s], 8);  // one arrival per softmax warp
+            mbar_init(&x.p_full[s], 8);
             mbar_init(&x.p_empty[s], 1);
         }
         mbar_init(&x.drain, 1);
         x.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == W_MMA) {
         tmem_alloc(&x.tmem_base, TMEM_COLS);
         tmem_relinquish();
+    }
+    if (tid < 64) x.m_s[tid >> 5][tid & 31] = -INFINITY;
+    for (int b = tid; b < min(cnt, ROWS_SMEM); b += ATTN_THREADS) {
+        int first;
+        x.rows[b] = static_cast<uint8_t>(block_rows(a, __ldg(lst + b), bh, &first));
     }
     // V slots are read in full by the PV MMA (M = 128 head-dim rows, K = 128
     // KV rows) even where a tile loads fewer rows; they start at zero so those
@@ -175,60 +236,50 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = x.tmem_base;
     volatile int* abort_flag = &x.abort;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == W_KPROD || warp == W_VPROD) {
+        // ------------------------------------------------------------ producers
         if (lane == 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
-            mbar_arrive_expect_tx(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
-            for (int p = 0; p < L::NP; ++p)
-                tma_load_2d(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
-            int k_armed = 0, v_armed = 0;  // tiles whose loads were issued
+            const bool is_k = warp == W_KPROD;
+            const int nslots = is_k ? KSLOTS : VSLOTS;
+            uint64_t* full = is_k ? x.k_full : x.v_full;
+            uint64_t* empty = is_k ? x.k_empty : x.v_empty;
+            uint8_t* base = smem + (is_k ? L::OFF_K : L::OFF_V);
+            const uint32_t slot_bytes = is_k ? L::K_SLOT : L::V_SLOT;
+            const CUtensorMap* mfull = is_k ? &tm_k : &tm_v;
+            const CUtensorMap* mpart = is_k ? &tm_k_rem : &tm_v_rem;
+            tma_prefetch_desc(mfull);
+            if (is_k) {
+                const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
+                mbar_arrive_expect_tx(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
+                for (int p = 0; p < L::NP; ++p)
+                    tma_load_2d(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
+            }
+            int armed = 0;  // tiles whose loads were issued
             for (int i = 0; i < n_tiles; ++i) {
                 const int nb = min(2, cnt - 2 * i);
                 int rows[2] = {0, 0}, first[2] = {0, 0};
                 for (int h = 0; h < nb; ++h) {
                     const int g = __ldg(lst + 2 * i + h);
                     rows[h] = block_rows(a, g, bh, &first[h]);
-                    if (rows[h] == 0) record_error(a.err, DEVERR_LIST | 2);
+                    if (rows[h] == 0 && is_k) record_error(a.err, DEVERR_LIST | 2);
                 }
                 const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NP);
-                const int ks = i % KSLOTS;
-                if (!mbar_wait(&x.k_empty[ks], ((i / KSLOTS) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
-                if (bytes) mbar_arrive_expect_tx(&x.k_full[ks], bytes);
-                else mbar_arrive(&x.k_full[ks]);
-                for (int h = 0; h < nb; ++h) {
-                    if (!rows[h]) continue;
-                    const CUtensorMap* m = rows[h] == 64 ? &tm_k : &tm_k_rem;
-                    for (int p = 0; p < L::NP; ++p)
-                        tma_load_2d(smem + L::OFF_K + ks * L::K_SLOT + p * L::PANEL_KV + h * 64 * 128, m,
-                                    p * 64, first[h], &x.k_full[ks]);
-                }
-                k_armed = i + 1;
-                const int vs = i % VSLOTS;
-                if (!mbar_wait(&x.v_empty[vs], ((i / VSLOTS) & 1) ^ 1, abort_flag, a.err, 0x11)) break;
-                if (bytes) mbar_arrive_expect_tx(&x.v_full[vs], bytes);
-                else mbar_arrive(&x.v_full[vs]);
-                for (int h = 0; h < nb; ++h) {
-                    if (!rows[h]) continue;
-                    const CUtensorMap* m = rows[h] == 64 ? &tm_v : &tm_v_rem;
-                    for (int p = 0; p < L::NP; ++p)
-                        tma_load_2d(smem + L::OFF_V + vs * L::V_SLOT + p * L::PANEL_KV + h * 64 * 128, m,
-                                    p * 64, first[h], &x.v_full[vs]);
-                }
-                v_armed = i + 1;
+                const int s = i % nslots;
+                if (!mbar_wait(&empty[s], ((i / nslots) & 1) ^ 1, abort_flag, a.err, is_k ? 0x10 : 0x11)) break;
+                if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
+                else mbar_arrive(&full[s]);
+                for (int h = 0; h < nb; ++h)
+                    if (rows[h]) load_block<D, IL>(base + s * slot_bytes, h, rows[h], first[h], mfull, mpart, &full[s]);
+                armed = i + 1;
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA exits.
-                mbar_drain(&x.q_full, 0, 10000000ull);
-                for (int i = max(0, k_armed - KSLOTS); i < k_armed; ++i)
-                    mbar_drain(&x.k_full[i % KSLOTS], (i / KSLOTS) & 1, 10000000ull);
-                for (int i = max(0, v_armed - VSLOTS); i < v_armed; ++i)
-                    mbar_drain(&x.v_full[i % VSLOTS], (i / VSLOTS) & 1, 10000000ull);
+                if (is_k) mbar_drain(&x.q_full, 0, 10000000ull);
+                for (int i = max(0, armed - nslots); i < armed; ++i)
+                    mbar_drain(&full[i % nslots], (i / nslots) & 1, 10000000ull);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
@@ -247,7 +298,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t panel = static_cast<uint32_t>(kk >> 2);
-                    const uint64_t ad = sdesc_sw128(sK + ks * L::K_SLOT + panel * L::PANEL_KV + (kk & 3) * 32, 16, 1024);
+                    // A = K tile (M = 128 KV rows, K-major), B = Q (N = 64 queries, K-major)
+                    const uint64_t ad =
+                        sdesc_sw128(sK + ks * L::K_SLOT + panel * L::KV_PANEL + (kk & 3) * 32, 16, L::KV_SBO);
                     const uint64_t bd = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
                     umma_bf16(d, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
                 }
@@ -259,6 +312,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (ok && n_tiles > 0) ok = issue_s(0);
             if (ok && n_tiles > 1) ok = issue_s(1);
             for (int i = 0; ok && i < n_tiles; ++i) {
+                // S buffer (i & 1) is free as soon as the softmax has read S_i:
+                // issue S_{i+2} then, so it runs while the softmax works on tile i.
+                if (i + 2 < n_tiles) {
+                    if (!mbar_wait(&x.s_free[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x24)) break;
+                    if (!issue_s(i + 2)) break;
+                }
                 if (!mbar_wait(&x.p_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x22)) break;
                 const int vs = i % VSLOTS;
                 if (!mbar_wait(&x.v_full[vs], (i / VSLOTS) & 1, abort_flag, a.err, 0x23)) break;
@@ -266,7 +325,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     // A = V^T (M = head_dim, MN-major: 64-wide panels LBO apart, 8-row K groups SBO apart)
-                    const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * 2048, L::PANEL_KV, 1024);
+                    const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * L::KV_K16, L::KV_PANEL, L::KV_SBO);
                     // B = P^T (N = 64 queries, MN-major, one 64-wide panel)
                     const uint64_t bd = sdesc_sw128(sP + (i & 1) * L::P_BUF + kk * 2048, L::P_BUF, 1024);
                     umma_bf16(tmem + 128, ad, bd, IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
@@ -274,41 +333,50 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 umma_commit(&x.v_empty[vs]);
                 umma_commit(&x.p_empty[i & 1]);
                 issued_any = true;
-                if (i + 2 < n_tiles && !issue_s(i + 2)) break;
             }
             if (*abort_flag && issued_any) {
                 umma_commit(&x.drain);
                 mbar_drain(&x.drain, 0, 10000000ull);
             }
         }
-    } else {
+    } else if (warp >= W_SOFT0) {
         // ------------------------------------------------------------ softmax
-        const int wg = (warp - 2) >> 2;        // query columns [32*wg, 32*wg + 32)
+        const int wg = (warp - W_SOFT0) >> 2;  // query columns [32*wg, 32*wg + 32)
         const int sp = warp & 3;               // TMEM sub-partition of this warp
         const int t = sp * 32 + lane;          // KV token of the tile / head-dim row of O^T
         const int bar_id = 1 + wg;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
         const uint32_t col0 = static_cast<uint32_t>(wg * 32);
         const float sl2 = a.scale_log2;
-        float m[32], l[32];
+        float l[32];  // this thread's share of each column's softmax denominator
 #pragma unroll
-        for (int c = 0; c < 32; ++c) { m[c] = -INFINITY; l[c] = 0.f; }
+        for (int c = 0; c < 32; ++c) l[c] = 0.f;
 
         for (int i = 0; i < n_tiles; ++i) {
-            const int hb = t >> 6;
-            const int bi = 2 * i + hb;
-            bool valid = false;
+            const int bi = 2 * i + (t >> 6);
+            int rows = 0;
             if (bi < cnt) {
-                int first;
-                const int rows = block_rows(a, __ldg(lst + bi), bh, &first);
-                valid = (t & 63) < rows;
+                if (bi < ROWS_SMEM) {
+                    rows = x.rows[bi];
+                } else {
+                    int first;
+                    rows = block_rows(a, __ldg(lst + bi), bh, &first);
+                }
             }
+            const bool valid = (t & 63) < rows;
+            const uint32_t s_addr = lane_base + static_cast<uint32_t>((i & 1) * 64) + col0;
             mbar_wait(&x.s_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x30);
             __syncwarp();
             tc_fence_after();
             float s[32];
-            tmem_ld32(lane_base + static_cast<uint32_t>((i & 1) * 64) + col0, s);
+            tmem_ld32(s_addr, s);
             tmem_ld_wait();
+            float m[32];
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+                const float4 t4 = *reinterpret_cast<const float4*>(&x.m_s[wg][c]);
+                m[c] = t4.x; m[c + 1] = t4.y; m[c + 2] = t4.z; m[c + 3] = t4.w;
+            }
             float xmax = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
@@ -317,23 +385,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             const bool need = named_bar_or(bar_id, 128, xmax > LAZY_RESCALE_LOG2);
             if (need) {
-                float v[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = s[c];
-                transpose_reduce<true>(v, lane);
-                x.red[wg][sp][lane] = v[0];
+                // Exact column maxima of this tile: butterfly within the warp
+                // (s is consumed and reloaded below), then across the 4 warps.
+                transpose_reduce<true>(s, lane);
+                x.red[wg][sp][lane] = s[0];
                 named_bar_sync(bar_id, 128);
-                float alpha[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float tmax = fmaxf(fmaxf(x.red[wg][0][c], x.red[wg][1][c]),
-                                             fmaxf(x.red[wg][2][c], x.red[wg][3][c]));
-                    const float mn = fmaxf(m[c], tmax);
-                    alpha[c] = (mn == -INFINITY) ? 1.f : fast_exp2(m[c] - mn);
-                    m[c] = mn;
-                    l[c] *= alpha[c];
-                }
+                // lane c owns column c: new stabiliser and rescale factor
+                const float m_old = x.m_s[wg][lane];
+                const float m_new = fmaxf(m_old, fmaxf(fmaxf(x.red[wg][0][lane], x.red[wg][1][lane]),
+                                                       fmaxf(x.red[wg][2][lane], x.red[wg][3][lane])));
+                const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_old - m_new);
                 named_bar_sync(bar_id, 128);
+                if (sp == 0) x.m_s[wg][lane] = m_new;
                 if (i > 0) {
                     // O^T columns of this warpgroup hold PV_0..PV_{i-1}: wait for
                     // PV_{i-2} (other P buffer) and PV_{i-1}, then rescale.
@@ -345,11 +408,32 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     tmem_ld32(lane_base + 128u + col0, o);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] *= alpha[c];
+                    for (int c = 0; c < 32; ++c) {
+                        const float ac = __shfl_sync(0xffffffffu, alpha, c);
+                        o[c] *= ac;
+                        l[c] *= ac;
+                    }
                     tmem_st32(lane_base + 128u + col0, o);
                     tmem_st_wait();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) l[c] *= __shfl_sync(0xffffffffu, alpha, c);
                 }
+                named_bar_sync(bar_id, 128);
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(&x.m_s[wg][c]);
+                    m[c] = t4.x; m[c + 1] = t4.y; m[c + 2] = t4.z; m[c + 3] = t4.w;
+                }
+                tmem_ld32(s_addr, s);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[c] = valid ? s[c] * sl2 : -INFINITY;
             }
+            // S_i is in registers: the MMA may overwrite this S buffer.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x.s_free[i & 1]);
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
@@ -371,7 +455,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&x.p_full[i & 1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x.p_full[i & 1]);
         }
 
         // ------------------------------------------------------------ epilogue
@@ -402,7 +487,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         named_bar_sync(3, 256);
         const int chunks = q_rows * (D / 8);
-        for (int idx = tid - 64; idx < chunks; idx += 256) {
+        for (int idx = tid - W_SOFT0 * 32; idx < chunks; idx += 256) {
             const int qq = idx / (D / 8);
             const int c8 = idx - qq * (D / 8);
             *reinterpret_cast<uint4*>(a.out + (static_cast<long long>(q_row0) + qq) * D + c8 * 8) =
@@ -412,35 +497,39 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
-template <int D>
-cudaError_t launch_attn_d(const AttnMaps& m, const AttnArgs& a, int n_rows, cudaStream_t s)
+template <int D, bool IL>
+cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, int n_rows, cudaStream_t s)
 {
-    constexpr uint32_t smem = attn_smem_bytes<D>();
+    constexpr uint32_t smem = attn_smem_bytes<D, IL>();
+    static_assert(smem <= 232448, "shared memory plan exceeds 227 KB");
     static int configured_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = cudaFuncSetAttribute(attn_kernel<D, IL>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    attn_kernel<D><<<static_cast<unsigned>(n_rows), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v, m.v_rem, a);
+    attn_kernel<D, IL><<<static_cast<unsigned>(n_rows), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
+                                                                               m.v_rem, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, int n_rows, cudaStream_t s)
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s)
 {
     if (n_rows <= 0) return cudaSuccess;
-    return D == 128 ? launch_attn_d<128>(m, a, n_rows, s) : launch_attn_d<64>(m, a, n_rows, s);
+    if (D == 128)
+        return interleaved ? launch_attn_t<128, true>(m, a, n_rows, s) : launch_attn_t<128, false>(m, a, n_rows, s);
+    return launch_attn_t<64, false>(m, a, n_rows, s);
 }
 
 }  // namespace lf

@@ -52,6 +52,7 @@ struct AttnMaps {
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s);
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s);
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, int n_rows, cudaStream_t s);
+// interleaved: K/V tensor maps are the 4-D block maps (head_dim 128 only).
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s);
 
 }  // namespace lf
