@@ -28,23 +28,27 @@
 //     loads (so a V slot that is still in use never delays K prefetch), warp 2
 //     allocates TMEM and issues tcgen05.mma from one thread, warp 3 idles,
 //     warps 4-11 are two softmax warpgroups. TMEM lane t of S^T is KV token t
-//     of the tile, so each softmax thread owns one KV token and 32 query
-//     columns (warpgroup 0: queries 0-31, warpgroup 1: queries 32-63).
+//     of the tile, so each softmax thread owns one KV token of a tile and all
+//     64 query columns.
+//   * Ping-pong. Warpgroup g takes the tiles i with i % 2 == g, with its own
+//     running maxima, its own O^T accumulator in TMEM and its own P buffer, so
+//     one warpgroup exponentiates while the other waits for its next scores;
+//     the two partial softmaxes are merged once in the epilogue
+//     (O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M))).
 //   * Online softmax in fp32, base 2, with a lazy stabiliser: each query
 //     column keeps m (running max of scale*log2(e)*score, in shared memory); a
 //     tile whose scores stay within m + 8 (p <= 256) is exponentiated against
 //     the current m with no cross-thread work; only when some score exceeds
 //     that bound does the warpgroup compute the exact column maxima of the tile
-//     (butterfly reductions + shared memory) and rescale its columns of O^T in
+//     (butterfly reductions + shared memory) and rescale its O^T columns in
 //     TMEM. Row sums are kept per thread and reduced once at the end.
 //   * P^T goes to shared memory as bf16 in the 128-byte-swizzled MN-major
 //     layout the MMA reads; masked KV tokens (past the end of a partial block,
 //     or the unused half of an odd last tile) get P = 0.
-//   * Pipelines: K ring of 3 slots, V ring of 2, S double-buffered in TMEM, P
-//     double-buffered in shared memory. The softmax releases an S buffer as
-//     soon as the scores are in registers, and the MMA thread then issues S
-//     for tile i+2 before PV for tile i, so the tensor pipe works on the next
-//     scores while the softmax exponentiates.
+//   * Pipelines: K ring of 3 slots, V ring of 2, four S buffers in TMEM (S is
+//     issued up to four tiles ahead), one P buffer per warpgroup. The MMA
+//     thread never blocks on one operand while another MMA is ready: it polls
+//     its barriers and issues whichever PV (first) or S is ready.
 //   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
@@ -64,7 +68,7 @@ constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_SOFT0 = 4;
 constexpr int KSLOTS = 3;
 constexpr int VSLOTS = 2;
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
-constexpr uint32_t TMEM_COLS = 256;         // S0: 0-63, S1: 64-127, O^T: 128-191
+constexpr uint32_t TMEM_COLS = 512;         // S buffers 0-3: columns 64*b; O^T of warpgroup g: 256 + 64*g
 constexpr int ROWS_SMEM = 1024;             // list entries whose row counts are cached in smem
 
 // Shared-memory plan. IL selects the interleaved K/V layout (head_dim 128,
@@ -95,12 +99,13 @@ struct AttnAux {
     uint64_t q_full;
     uint64_t k_full[KSLOTS], k_empty[KSLOTS];
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
-    uint64_t s_full[2], s_free[2], p_full[2], p_empty[2];
+    uint64_t s_full[4], s_free[4], p_full[2], p_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    float red[2][4][32];
-    alignas(16) float m_s[2][32];  // running max (log2 units) of each query column (read as float4)
+    float red[2][4][64];
+    float lsum[2][64];             // softmax denominators of each warpgroup's columns
+    alignas(16) float m_s[2][64];  // running max (log2 units) per warpgroup and query column (read as float4)
     uint8_t rows[ROWS_SMEM];       // valid token rows of list entry b (0: not a valid block)
 };
 
@@ -197,10 +202,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(&x.q_full, 1);
         for (int s = 0; s < KSLOTS; ++s) { mbar_init(&x.k_full[s], 1); mbar_init(&x.k_empty[s], 1); }
         for (int s = 0; s < VSLOTS; ++s) { mbar_init(&x.v_full[s], 1); mbar_init(&x.v_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 4; ++s) {
             mbar_init(&x.s_full[s], 1);
-            mbar_init(&x.s_free[s], 8);  // one arrival per softmax warp
-            mbar_init(&x.p_full[s], 8);
+            mbar_init(&x.s_free[s], 4);  // one arrival per warp of the owning warpgroup
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&x.p_full[s], 4);
             mbar_init(&x.p_empty[s], 1);
         }
         mbar_init(&x.drain, 1);
@@ -211,7 +218,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_alloc(&x.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
-    if (tid < 64) x.m_s[tid >> 5][tid & 31] = -INFINITY;
+    if (tid < 128) x.m_s[tid >> 6][tid & 63] = -INFINITY;
     for (int b = tid; b < min(cnt, ROWS_SMEM); b += ATTN_THREADS) {
         int first;
         x.rows[b] = static_cast<uint8_t>(block_rows(a, __ldg(lst + b), bh, &first));
@@ -290,49 +297,65 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const uint32_t sP = smem_u32(smem + L::OFF_P);
             bool issued_any = false;
             bool ok = mbar_wait(&x.q_full, 0, abort_flag, a.err, 0x20);
-            auto issue_s = [&](int j) -> bool {
-                const int ks = j % KSLOTS;
-                if (!mbar_wait(&x.k_full[ks], (j / KSLOTS) & 1, abort_flag, a.err, 0x21)) return false;
-                tc_fence_after();
-                const uint32_t d = tmem + static_cast<uint32_t>((j & 1) * 64);
+            int next_s = 0, next_pv = 0;
+            unsigned long long stall_t0 = 0;
+            uint32_t idle = 0;
+            while (ok && next_pv < n_tiles) {
+                bool progressed = false;
+                // PV for the oldest tile whose P and V are ready (frees a V slot and a P buffer).
+                if (next_pv < next_s) {
+                    const int i = next_pv, g = i & 1, vs = i % VSLOTS;
+                    if (mbar_test(&x.p_full[g], (i >> 1) & 1) && mbar_test(&x.v_full[vs], (i / VSLOTS) & 1)) {
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t panel = static_cast<uint32_t>(kk >> 2);
-                    // A = K tile (M = 128 KV rows, K-major), B = Q (N = 64 queries, K-major)
-                    const uint64_t ad =
-                        sdesc_sw128(sK + ks * L::K_SLOT + panel * L::KV_PANEL + (kk & 3) * 32, 16, L::KV_SBO);
-                    const uint64_t bd = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
-                    umma_bf16(d, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            // A = V^T (M = head_dim, MN-major: 64-wide panels LBO apart, 8-row K groups SBO apart)
+                            const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * L::KV_K16, L::KV_PANEL, L::KV_SBO);
+                            // B = P^T (N = 64 queries, MN-major, one 64-wide panel)
+                            const uint64_t bd = sdesc_sw128(sP + g * L::P_BUF + kk * 2048, L::P_BUF, 1024);
+                            umma_bf16(tmem + 256u + 64u * g, ad, bd, IDESC_O, (i >= 2 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&x.v_empty[vs]);
+                        umma_commit(&x.p_empty[g]);
+                        issued_any = true;
+                        ++next_pv;
+                        progressed = true;
+                    }
                 }
-                umma_commit(&x.k_empty[ks]);
-                umma_commit(&x.s_full[j & 1]);
-                issued_any = true;
-                return true;
-            };
-            if (ok && n_tiles > 0) ok = issue_s(0);
-            if (ok && n_tiles > 1) ok = issue_s(1);
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                // S buffer (i & 1) is free as soon as the softmax has read S_i:
-                // issue S_{i+2} then, so it runs while the softmax works on tile i.
-                if (i + 2 < n_tiles) {
-                    if (!mbar_wait(&x.s_free[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x24)) break;
-                    if (!issue_s(i + 2)) break;
-                }
-                if (!mbar_wait(&x.p_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x22)) break;
-                const int vs = i % VSLOTS;
-                if (!mbar_wait(&x.v_full[vs], (i / VSLOTS) & 1, abort_flag, a.err, 0x23)) break;
-                tc_fence_after();
+                // S for the next tile once its TMEM buffer is free and its K has landed.
+                if (next_s < n_tiles) {
+                    const int i = next_s, b = i & 3, ks = i % KSLOTS;
+                    const bool buf_free = i < 4 || mbar_test(&x.s_free[b], ((i >> 2) - 1) & 1);
+                    if (buf_free && mbar_test(&x.k_full[ks], (i / KSLOTS) & 1)) {
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // A = V^T (M = head_dim, MN-major: 64-wide panels LBO apart, 8-row K groups SBO apart)
-                    const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * L::KV_K16, L::KV_PANEL, L::KV_SBO);
-                    // B = P^T (N = 64 queries, MN-major, one 64-wide panel)
-                    const uint64_t bd = sdesc_sw128(sP + (i & 1) * L::P_BUF + kk * 2048, L::P_BUF, 1024);
-                    umma_bf16(tmem + 128, ad, bd, IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t panel = static_cast<uint32_t>(kk >> 2);
+                            // A = K tile (M = 128 KV rows, K-major), B = Q (N = 64 queries, K-major)
+                            const uint64_t ad =
+                                sdesc_sw128(sK + ks * L::K_SLOT + panel * L::KV_PANEL + (kk & 3) * 32, 16, L::KV_SBO);
+                            const uint64_t bd = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
+                            umma_bf16(tmem + 64u * b, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&x.k_empty[ks]);
+                        umma_commit(&x.s_full[b]);
+                        issued_any = true;
+                        ++next_s;
+                        progressed = true;
+                    }
                 }
-                umma_commit(&x.v_empty[vs]);
-                umma_commit(&x.p_empty[i & 1]);
-                issued_any = true;
+                if (progressed) {
+                    idle = 0;
+                } else if (++idle == 1) {
+                    stall_t0 = globaltimer();
+                } else if ((idle & 63u) == 0u) {
+                    if (*abort_flag) break;
+                    if (globaltimer() - stall_t0 > LF_WAIT_LIMIT_NS) {
+                        *abort_flag = 1;
+                        record_error(a.err, DEVERR_TIMEOUT | 0x22);
+                        break;
+                    }
+                }
             }
             if (*abort_flag && issued_any) {
                 umma_commit(&x.drain);
@@ -341,18 +364,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     } else if (warp >= W_SOFT0) {
         // ------------------------------------------------------------ softmax
-        const int wg = (warp - W_SOFT0) >> 2;  // query columns [32*wg, 32*wg + 32)
+        const int g = (warp - W_SOFT0) >> 2;   // this warpgroup takes the tiles i with i % 2 == g
         const int sp = warp & 3;               // TMEM sub-partition of this warp
-        const int t = sp * 32 + lane;          // KV token of the tile / head-dim row of O^T
-        const int bar_id = 1 + wg;
+        const int t = sp * 32 + lane;          // KV token of a tile / head-dim row of O^T
+        const int bar_id = 1 + g;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
-        const uint32_t col0 = static_cast<uint32_t>(wg * 32);
+        const uint32_t o_col = 256u + 64u * static_cast<uint32_t>(g);
         const float sl2 = a.scale_log2;
-        float l[32];  // this thread's share of each column's softmax denominator
+        uint8_t* pbuf = smem + L::OFF_P + g * L::P_BUF + (t >> 3) * 1024 + (t & 7) * 128;
+        float l[64];  // this thread's share of each column's softmax denominator
 #pragma unroll
-        for (int c = 0; c < 32; ++c) l[c] = 0.f;
+        for (int c = 0; c < 64; ++c) l[c] = 0.f;
 
-        for (int i = 0; i < n_tiles; ++i) {
+        for (int i = g; i < n_tiles; i += 2) {
+            const int j = i >> 1;  // local tile index of this warpgroup
             const int bi = 2 * i + (t >> 6);
             int rows = 0;
             if (bi < cnt) {
@@ -364,125 +389,167 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
             const bool valid = (t & 63) < rows;
-            const uint32_t s_addr = lane_base + static_cast<uint32_t>((i & 1) * 64) + col0;
-            mbar_wait(&x.s_full[i & 1], (i >> 1) & 1, abort_flag, a.err, 0x30);
+            const uint32_t s_addr = lane_base + 64u * static_cast<uint32_t>(i & 3);
+            mbar_wait(&x.s_full[i & 3], (i >> 2) & 1, abort_flag, a.err, 0x30);
             __syncwarp();
             tc_fence_after();
-            float s[32];
-            tmem_ld32(s_addr, s);
-            tmem_ld_wait();
-            float m[32];
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-                const float4 t4 = *reinterpret_cast<const float4*>(&x.m_s[wg][c]);
-                m[c] = t4.x; m[c + 1] = t4.y; m[c + 2] = t4.z; m[c + 3] = t4.w;
-            }
+            // 1. Does any score exceed the stabiliser by more than the lazy bound?
             float xmax = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                s[c] = valid ? s[c] * sl2 : -INFINITY;
-                xmax = fmaxf(xmax, s[c] - m[c]);
-            }
-            const bool need = named_bar_or(bar_id, 128, xmax > LAZY_RESCALE_LOG2);
-            if (need) {
-                // Exact column maxima of this tile: butterfly within the warp
-                // (s is consumed and reloaded below), then across the 4 warps.
-                transpose_reduce<true>(s, lane);
-                x.red[wg][sp][lane] = s[0];
-                named_bar_sync(bar_id, 128);
-                // lane c owns column c: new stabiliser and rescale factor
-                const float m_old = x.m_s[wg][lane];
-                const float m_new = fmaxf(m_old, fmaxf(fmaxf(x.red[wg][0][lane], x.red[wg][1][lane]),
-                                                       fmaxf(x.red[wg][2][lane], x.red[wg][3][lane])));
-                const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_old - m_new);
-                named_bar_sync(bar_id, 128);
-                if (sp == 0) x.m_s[wg][lane] = m_new;
-                if (i > 0) {
-                    // O^T columns of this warpgroup hold PV_0..PV_{i-1}: wait for
-                    // PV_{i-2} (other P buffer) and PV_{i-1}, then rescale.
-                    mbar_wait(&x.p_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag, a.err, 0x31);
-                    mbar_wait(&x.p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.err, 0x32);
-                    __syncwarp();
-                    tc_fence_after();
-                    float o[32];
-                    tmem_ld32(lane_base + 128u + col0, o);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float ac = __shfl_sync(0xffffffffu, alpha, c);
-                        o[c] *= ac;
-                        l[c] *= ac;
-                    }
-                    tmem_st32(lane_base + 128u + col0, o);
-                    tmem_st_wait();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) l[c] *= __shfl_sync(0xffffffffu, alpha, c);
-                }
-                named_bar_sync(bar_id, 128);
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(&x.m_s[wg][c]);
-                    m[c] = t4.x; m[c + 1] = t4.y; m[c + 2] = t4.z; m[c + 3] = t4.w;
-                }
-                tmem_ld32(s_addr, s);
+            for (int h = 0; h < 2; ++h) {
+                float s[32];
+                tmem_ld32(s_addr + 32u * h, s);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[c] = valid ? s[c] * sl2 : -INFINITY;
-            }
-            // S_i is in registers: the MMA may overwrite this S buffer.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&x.s_free[i & 1]);
-            uint32_t pk[16];
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(&x.m_s[g][32 * h + c]);
+                    s[c] = fmaf(s[c], sl2, -m4.x);
+                    s[c + 1] = fmaf(s[c + 1], sl2, -m4.y);
+                    s[c + 2] = fmaf(s[c + 2], sl2, -m4.z);
+                    s[c + 3] = fmaf(s[c + 3], sl2, -m4.w);
+                }
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                const float p0 = valid ? fast_exp2(s[c] - m[c]) : 0.f;
-                const float p1 = valid ? fast_exp2(s[c + 1] - m[c + 1]) : 0.f;
-                l[c] += p0;
-                l[c + 1] += p1;
-                pk[c >> 1] = pack_bf16x2(p0, p1);
-            }
-            // P buffer (i & 1) was last read by PV_{i-2}.
-            if (i >= 2) mbar_wait(&x.p_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag, a.err, 0x33);
-            __syncwarp();
-            uint8_t* prow = smem + L::OFF_P + (i & 1) * L::P_BUF + (t >> 3) * 1024 + (t & 7) * 128;
+                for (int w = 16; w >= 1; w >>= 1)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int chunk = (wg * 4 + k) ^ (t & 7);
-                *reinterpret_cast<uint4*>(prow + chunk * 16) =
-                    make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                    for (int c = 0; c < w; ++c) s[c] = fmaxf(s[c], s[c + w]);
+                xmax = fmaxf(xmax, s[0]);
+            }
+            if (!valid) xmax = -INFINITY;
+            const bool need = named_bar_or(bar_id, 128, xmax > LAZY_RESCALE_LOG2);
+            // PV of this warpgroup's previous tile must be done before its P
+            // buffer is rewritten or its O^T columns are rescaled.
+            if (j > 0) mbar_wait(&x.p_empty[g], (j - 1) & 1, abort_flag, a.err, 0x31);
+            __syncwarp();
+            if (need) {
+                // 2. Exact column maxima of this tile over its 128 KV tokens.
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float s[32];
+                    tmem_ld32(s_addr + 32u * h, s);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) s[c] = valid ? s[c] * sl2 : -INFINITY;
+                    transpose_reduce<true>(s, lane);
+                    x.red[g][sp][32 * h + lane] = s[0];
+                }
+                named_bar_sync(bar_id, 128);
+                float alpha[2], m_new[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 32 * h + lane;  // lane owns column c of this half
+                    const float m_old = x.m_s[g][c];
+                    m_new[h] = fmaxf(m_old, fmaxf(fmaxf(x.red[g][0][c], x.red[g][1][c]),
+                                                  fmaxf(x.red[g][2][c], x.red[g][3][c])));
+                    alpha[h] = (m_new[h] == -INFINITY) ? 1.f : fast_exp2(m_old - m_new[h]);
+                }
+                named_bar_sync(bar_id, 128);  // every warp has read the old maxima
+                if (sp == 0) {
+                    x.m_s[g][lane] = m_new[0];
+                    x.m_s[g][32 + lane] = m_new[1];
+                }
+                tc_fence_after();
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (j > 0) {
+                        float o[32];
+                        tmem_ld32(lane_base + o_col + 32u * h, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] *= __shfl_sync(0xffffffffu, alpha[h], c);
+                        tmem_st32(lane_base + o_col + 32u * h, o);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) l[32 * h + c] *= __shfl_sync(0xffffffffu, alpha[h], c);
+                }
+                if (j > 0) tmem_st_wait();
+                named_bar_sync(bar_id, 128);
+            }
+            // 3. Probabilities P = 2^(s*scale*log2e - m) as bf16 P^T rows.
+            __syncwarp();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float s[32];
+                tmem_ld32(s_addr + 32u * h, s);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(&x.m_s[g][32 * h + c]);
+                    const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; e += 2) {
+                        const float p0 = valid ? fast_exp2(fmaf(s[c + e], sl2, -mm[e])) : 0.f;
+                        const float p1 = valid ? fast_exp2(fmaf(s[c + e + 1], sl2, -mm[e + 1])) : 0.f;
+                        l[32 * h + c + e] += p0;
+                        l[32 * h + c + e + 1] += p1;
+                        pk[(c + e) >> 1] = pack_bf16x2(p0, p1);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int chunk = (4 * h + k) ^ (t & 7);
+                    *reinterpret_cast<uint4*>(pbuf + chunk * 16) =
+                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&x.p_full[i & 1]);
+            if (lane == 0) {
+                mbar_arrive(&x.s_free[i & 3]);
+                mbar_arrive(&x.p_full[g]);
+            }
         }
 
         // ------------------------------------------------------------ epilogue
-        if (n_tiles > 0)
-            mbar_wait(&x.p_empty[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, a.err, 0x34);
+        const int n_g = (n_tiles - g + 1) >> 1;  // tiles this warpgroup took
+        if (n_g > 0) mbar_wait(&x.p_empty[g], (n_g - 1) & 1, abort_flag, a.err, 0x34);
         __syncwarp();
         tc_fence_after();
-        transpose_reduce<false>(l, lane);
-        x.red[wg][sp][lane] = l[0];
-        named_bar_sync(bar_id, 128);
-        float o[32];
-        if (n_tiles > 0) {
-            tmem_ld32(lane_base + 128u + col0, o);
-            tmem_ld_wait();
-        } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        for (int h = 0; h < 2; ++h) {
+            float v[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = l[32 * h + c];
+            transpose_reduce<false>(v, lane);
+            x.red[g][sp][32 * h + lane] = v[0];
         }
-        // Stage O (bf16, [query][head_dim]) in the K ring, free now.
+        named_bar_sync(bar_id, 128);
+        if (sp == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = 32 * h + lane;
+                x.lsum[g][c] = x.red[g][0][c] + x.red[g][1][c] + x.red[g][2][c] + x.red[g][3][c];
+            }
+        }
+        tc_fence_before();
+        named_bar_sync(3, 256);  // both warpgroups: sums, maxima and last PVs are final
+        tc_fence_after();
+        // Warpgroup g merges and writes query columns [32g, 32g + 32).
+        const int n0 = (n_tiles + 1) >> 1, n1 = n_tiles >> 1;
+        float o0[32], o1[32];
+        __syncwarp();
+        if (n0 > 0) {
+            tmem_ld32(lane_base + 256u + 32u * g, o0);
+        }
+        if (n1 > 0) {
+            tmem_ld32(lane_base + 320u + 32u * g, o1);
+        }
+        tmem_ld_wait();
         __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K);
         if (t < D) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const float lsum = x.red[wg][0][c] + x.red[wg][1][c] + x.red[wg][2][c] + x.red[wg][3][c];
-                const float val = lsum > 0.f ? o[c] / lsum : 0.f;
-                ostage[(col0 + c) * D + t] = __float2bfloat16_rn(val);
+                const int cc = 32 * g + c;
+                const float m0 = x.m_s[0][cc], m1 = x.m_s[1][cc];
+                const float mx = fmaxf(m0, m1);
+                const float f0 = (n0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - mx) : 0.f;
+                const float f1 = (n1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - mx) : 0.f;
+                const float den = x.lsum[0][cc] * f0 + x.lsum[1][cc] * f1;
+                const float num = (f0 != 0.f ? o0[c] * f0 : 0.f) + (f1 != 0.f ? o1[c] * f1 : 0.f);
+                ostage[cc * D + t] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
             }
         }
         named_bar_sync(3, 256);
