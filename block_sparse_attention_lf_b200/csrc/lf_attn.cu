@@ -7,48 +7,42 @@
 //   * One CTA per query block (64 query tokens of one head, its own KV block
 //     list). CTAs are ordered head-major so a head's K/V stay L2-resident while
 //     its query blocks run.
-//   * KV-major formulation. A tile is two listed KV blocks (128 tokens). The
-//     tensor core computes S^T = K_tile * Q^T (M = 128 KV tokens, N = 64
-//     queries, K = head_dim) into TMEM, and O^T += V_tile^T * P^T (M = 128
-//     head-dim rows, N = 64 queries, K = 128 KV tokens). Both MMAs run with
-//     M = 128 (M = 64 issues at half rate on this part) on exactly the listed
-//     blocks, with no union of neighbouring query blocks' lists.
-//   * Gather. K and V dominate the traffic (each query block reads its own
-//     ~100 blocks from L2). Small TMA boxes cap the per-SM L2 bandwidth, so
-//     for head_dim 128 each 64-token block (16 KB, contiguous) arrives as ONE
-//     4-D box {64 elems, 8 rows, 2 panels, 8 row groups} that lands in an
-//     interleaved layout [row group][panel][8 rows x 128 B] (128-byte swizzle).
-//     Its 8-row groups sit a uniform 2 KB apart, so one smem descriptor spans
-//     both blocks of a tile for the S^T MMA (SBO = 2 KB, panel at +1 KB) and
-//     for the PV MMA (MN-major: LBO = 1 KB between head-dim panels, SBO = 2 KB
-//     between 8-row groups). Frames whose token count is not a multiple of 8,
-//     and head_dim 64, use 2-D boxes per 64-wide panel into a plain
-//     [panel][row] layout instead.
+//   * A tile is two listed KV blocks (128 tokens); a step is two tiles. The
+//     scores of a step are two M = 64 MMAs, S_h = Q * K_tile(h)^T (M = 64
+//     queries, N = 128 keys, K = head_dim), written to the two halves of the
+//     TMEM lanes: query row r of tile h lands in lane 32*(r/16) + 16*h + r%16.
+//     A softmax thread therefore owns one query row of one tile, so row maxima
+//     and row sums need no cross-thread reduction (the two threads of a row,
+//     lanes l and l^16, exchange one value per step).
+//   * P goes to shared memory as bf16 in the 128-byte-swizzled K-major layout
+//     of the PV MMA's B operand, and O^T += V_block^T * P^T runs KV-major
+//     (M = 128 head-dim rows, N = 64 queries, K = 16 keys per instruction),
+//     which keeps that MMA at M = 128 (M = 64 issues at half rate).
+//   * Gather. For head_dim 128 each 64-token block (16 KB, contiguous) arrives
+//     as ONE 4-D TMA box {64 elems, 8 rows, 2 panels, 8 row groups} that lands
+//     in an interleaved layout [row group][panel][8 rows x 128 B] (128-byte
+//     swizzle) with a uniform 2 KB row-group stride, so one descriptor spans a
+//     tile's two blocks (K, SBO = 2 KB, panel at +1 KB) and a V block is read
+//     MN-major (LBO = 1 KB between head-dim panels, SBO = 2 KB between 8-row
+//     groups). Frames whose token count is not a multiple of 8, and head_dim
+//     64, use 2-D boxes per 64-wide panel into a plain [panel][row] layout.
+//     K arrives per tile (ring of 3 tiles), V per block (ring of 4 blocks).
 //   * Warp roles (384 threads): warp 0 issues the Q and K loads, warp 1 the V
-//     loads (so a V slot that is still in use never delays K prefetch), warp 2
-//     allocates TMEM and issues tcgen05.mma from one thread, warp 3 idles,
-//     warps 4-11 are two softmax warpgroups. TMEM lane t of S^T is KV token t
-//     of the tile, so each softmax thread owns one KV token of a tile and all
-//     64 query columns.
-//   * Ping-pong. Warpgroup g takes the tiles i with i % 2 == g, with its own
-//     running maxima, its own O^T accumulator in TMEM and its own P buffer, so
-//     one warpgroup exponentiates while the other waits for its next scores;
-//     the two partial softmaxes are merged once in the epilogue
-//     (O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M))).
-//   * Online softmax in fp32, base 2, with a lazy stabiliser: each query
-//     column keeps m (running max of scale*log2(e)*score, in shared memory); a
-//     tile whose scores stay within m + 8 (p <= 256) is exponentiated against
-//     the current m with no cross-thread work; only when some score exceeds
-//     that bound does the warpgroup compute the exact column maxima of the tile
-//     (butterfly reductions + shared memory) and rescale its O^T columns in
-//     TMEM. Row sums are kept per thread and reduced once at the end.
-//   * P^T goes to shared memory as bf16 in the 128-byte-swizzled MN-major
-//     layout the MMA reads; masked KV tokens (past the end of a partial block,
-//     or the unused half of an odd last tile) get P = 0.
-//   * Pipelines: K ring of 3 slots, V ring of 2, four S buffers in TMEM (S is
-//     issued up to four tiles ahead), one P buffer per warpgroup. The MMA
-//     thread never blocks on one operand while another MMA is ready: it polls
-//     its barriers and issues whichever PV (first) or S is ready.
+//     loads, warp 2 allocates TMEM and issues tcgen05.mma from one thread,
+//     warp 3 idles, warps 4-11 are two softmax warpgroups. Warpgroup g takes
+//     the steps s with s % 2 == g, with its own running maxima and its own O^T
+//     accumulator in TMEM; the two partial softmaxes are merged once in the
+//     epilogue (O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M))).
+//   * Online softmax in fp32, base 2, with a lazy stabiliser: each query row
+//     keeps m (running max of scale*log2(e)*score); a step whose scores stay
+//     within m + 8 (p <= 256) is exponentiated against the current m; only when
+//     some row exceeds that bound does the warpgroup move m and rescale the
+//     matching O^T columns in TMEM.
+//   * Pipelines: three S buffers in TMEM (S runs up to three steps ahead), one
+//     P buffer (the warpgroups write it in step order), per-block V release.
+//     The MMA thread never blocks on one operand while another MMA is ready: it
+//     polls its barriers and issues whichever PV block (first) or S tile is
+//     ready.
 //   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
@@ -65,33 +59,39 @@ namespace {
 
 constexpr int ATTN_THREADS = 384;
 constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_SOFT0 = 4;
-constexpr int KSLOTS = 3;
-constexpr int VSLOTS = 2;
+constexpr int KSLOTS = 3;   // K ring: tiles of two blocks
+constexpr int VSLOTS = 4;   // V ring: single blocks
+constexpr int SBUFS = 3;    // S buffers in TMEM (one per step in flight)
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
-constexpr uint32_t TMEM_COLS = 512;         // S buffers 0-3: columns 64*b; O^T of warpgroup g: 256 + 64*g
-constexpr int ROWS_SMEM = 1024;             // list entries whose row counts are cached in smem
+constexpr uint32_t TMEM_COLS = 512;         // S buffer b: columns 128*b; O^T of warpgroup g: 384 + 64*g
+constexpr uint32_t TM_O = 384;
+constexpr int LIST_SMEM = 1024;             // list entries staged in shared memory
 
 // Shared-memory plan. IL selects the interleaved K/V layout (head_dim 128,
-// one 4-D box per block); otherwise K/V use [panel][128 rows x 128 B].
+// one 4-D box per block); otherwise K/V use [panel][rows x 128 B].
 template <int D, bool IL>
 struct AttnLayout {
-    static constexpr int NP = D / 64;                  // 64-element panels of head_dim
-    static constexpr uint32_t PANEL_Q = 64u * 128u;     // 64 rows x 128 B
-    static constexpr uint32_t PANEL_KV = 128u * 128u;   // 128 rows x 128 B (panel layout)
-    static constexpr uint32_t BLOCK_IL = 16384u;        // one 64 x 128 bf16 block (interleaved)
+    static constexpr int NP = D / 64;                    // 64-element panels of head_dim
+    static constexpr uint32_t PANEL_Q = 64u * 128u;       // 64 rows x 128 B
+    static constexpr uint32_t BLOCK_IL = 16384u;          // one 64 x 128 bf16 block (interleaved)
     static constexpr uint32_t Q_BYTES = NP * PANEL_Q;
-    static constexpr uint32_t K_SLOT = NP * PANEL_KV;
-    static constexpr uint32_t V_SLOT = 2u * PANEL_KV;   // the PV MMA has M = 128 head-dim rows
-    static constexpr uint32_t P_BUF = 128u * 128u;      // P^T: 128 KV rows x 64 queries bf16
+    static constexpr uint32_t K_SLOT = NP * 128u * 128u;  // a tile: 128 rows
+    static constexpr uint32_t V_SLOT = 2u * 64u * 128u;   // a block; the PV MMA has M = 128 head-dim rows
+    static constexpr uint32_t P_PANEL = 64u * 128u;       // 64 queries x 64 keys bf16
+    static constexpr uint32_t P_BYTES = 4u * P_PANEL;     // a step: 256 keys
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + KSLOTS * K_SLOT;
     static constexpr uint32_t OFF_P = OFF_V + VSLOTS * V_SLOT;
-    static constexpr uint32_t OFF_AUX = OFF_P + 2u * P_BUF;
-    // smem descriptor strides of the K/V tiles
-    static constexpr uint32_t KV_SBO = IL ? 2048u : 1024u;          // between 8-row groups
-    static constexpr uint32_t KV_PANEL = IL ? 1024u : PANEL_KV;     // between 64-wide panels
-    static constexpr uint32_t KV_K16 = IL ? 4096u : 2048u;          // 16 KV rows (one PV k-step)
+    static constexpr uint32_t OFF_AUX = OFF_P + P_BYTES;
+    // K tile (B operand of the S MMA, K-major): 8-row group stride and panel offset
+    static constexpr uint32_t K_SBO = IL ? 2048u : 1024u;
+    static constexpr uint32_t K_PANEL = IL ? 1024u : 128u * 128u;
+    // V block (A operand of the PV MMA, MN-major): head-dim panel stride (LBO),
+    // 8-row group stride (SBO), and the step between 16-key k-slices
+    static constexpr uint32_t V_LBO = IL ? 1024u : 64u * 128u;
+    static constexpr uint32_t V_SBO = IL ? 2048u : 1024u;
+    static constexpr uint32_t V_K16 = IL ? 4096u : 2048u;
     static_assert(!IL || D == 128, "interleaved layout is for head_dim 128");
 };
 
@@ -99,38 +99,23 @@ struct AttnAux {
     uint64_t q_full;
     uint64_t k_full[KSLOTS], k_empty[KSLOTS];
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
-    uint64_t s_full[4], s_free[4], p_full[2], p_empty[2];
+    uint64_t s_full[SBUFS], s_free[SBUFS];
+    uint64_t p_full, p_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    float red[2][4][64];
-    float lsum[2][64];             // softmax denominators of each warpgroup's columns
-    alignas(16) float m_s[2][64];  // running max (log2 units) per warpgroup and query column (read as float4)
-    uint8_t rows[ROWS_SMEM];       // valid token rows of list entry b (0: not a valid block)
+    alignas(16) float alpha[2][64];  // per-warpgroup rescale factors of the query columns
+    float lsum[2][64];               // softmax denominators of each warpgroup's rows
+    alignas(16) float m_s[2][64];    // final running max (log2 units) per warpgroup and query row
+    int lst[LIST_SMEM];              // the CTA's block list (entries past LIST_SMEM stay in global memory)
 };
 
-static_assert(offsetof(AttnAux, m_s) % 16 == 0, "m_s is read with 16-byte loads");
+static_assert(offsetof(AttnAux, alpha) % 16 == 0, "alpha is read with 16-byte loads");
 
 template <int D, bool IL>
 constexpr uint32_t attn_smem_bytes()
 {
     return AttnLayout<D, IL>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux)) + 1024u;
-}
-
-template <bool MAX>
-__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane)
-{
-#pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
-        const bool upper = (lane & s) != 0;
-#pragma unroll
-        for (int i = 0; i < s; ++i) {
-            const float send = upper ? v[i] : v[i + s];
-            const float keep = upper ? v[i + s] : v[i];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, s);
-            v[i] = MAX ? fmaxf(keep, recv) : keep + recv;
-        }
-    }
 }
 
 // Token rows of KV block g (0 when g is not a valid block id) and its first
@@ -144,29 +129,58 @@ __device__ __forceinline__ int block_rows(const AttnArgs& a, int g, int bh, int*
     return (j == a.bpf - 1) ? a.rem : 64;
 }
 
-__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                            uint64_t* bar)
+// List entry b, from the shared-memory copy when it holds it.
+__device__ __forceinline__ int list_entry(const int* lst_s, const int* lst, int b)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-        : "memory");
+    return b < LIST_SMEM ? lst_s[b] : __ldg(lst + b);
+}
+
+// Valid rows of list entry b (0 past the end of the list or for a bad id).
+__device__ __forceinline__ int entry_rows(const AttnArgs& a, const int* lst_s, const int* lst, int b, int cnt)
+{
+    if (b >= cnt) return 0;
+    const int g = list_entry(lst_s, lst, b);
+    if (g < 0 || g >= a.Nkv) return 0;
+    return (g % a.bpf == a.bpf - 1) ? a.rem : 64;
 }
 
 // Load one KV block (`rows` valid tokens starting at flattened row `first`)
-// into half `h` of a K or V slot.
+// to `dst`; `panel_stride` separates the 64-wide panels of the plain layout.
+// Called by a converged producer warp; one elected lane issues the copies.
 template <int D, bool IL>
-__device__ __forceinline__ void load_block(uint8_t* slot, int h, int rows, int first, const CUtensorMap* full,
-                                           const CUtensorMap* part, uint64_t* bar)
+__device__ __forceinline__ void load_block(uint8_t* dst, uint32_t panel_stride, int rows, int first,
+                                           const CUtensorMap* full, const CUtensorMap* part, uint64_t* bar)
 {
     using L = AttnLayout<D, IL>;
     const CUtensorMap* m = rows == 64 ? full : part;
     if constexpr (IL) {
-        tma_load_4d(slot + h * L::BLOCK_IL, m, 0, 0, 0, first >> 3, bar);
+        tma_load_4d_elect(dst, m, 0, 0, 0, first >> 3, bar);
     } else {
 #pragma unroll
-        for (int p = 0; p < L::NP; ++p) tma_load_2d(slot + p * L::PANEL_KV + h * 64 * 128, m, p * 64, first, bar);
+        for (int p = 0; p < L::NP; ++p) tma_load_2d_elect(dst + p * panel_stride, m, p * 64, first, bar);
+    }
+}
+
+// 128 consecutive fp32 columns of this thread's TMEM lane (issued as four
+// loads; the caller waits).
+__device__ __forceinline__ void tmem_ld128_nowait(uint32_t taddr, float (&v)[128])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+              "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+              "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+              "=r"(r[31])
+            : "r"(taddr + 32u * q));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[32 * q + i] = __uint_as_float(r[i]);
     }
 }
 
@@ -193,6 +207,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     const int* lst = a.block_list + static_cast<long long>(row) * a.list_cap;
     const int n_tiles = (cnt + 1) >> 1;
+    const int n_steps = (n_tiles + 1) >> 1;
     const int fq = r / a.bpf;
     const int jq = r - fq * a.bpf;
     const int q_rows = (jq == a.bpf - 1) ? a.rem : 64;
@@ -202,14 +217,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(&x.q_full, 1);
         for (int s = 0; s < KSLOTS; ++s) { mbar_init(&x.k_full[s], 1); mbar_init(&x.k_empty[s], 1); }
         for (int s = 0; s < VSLOTS; ++s) { mbar_init(&x.v_full[s], 1); mbar_init(&x.v_empty[s], 1); }
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 0; s < SBUFS; ++s) {
             mbar_init(&x.s_full[s], 1);
             mbar_init(&x.s_free[s], 4);  // one arrival per warp of the owning warpgroup
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&x.p_full[s], 4);
-            mbar_init(&x.p_empty[s], 1);
-        }
+        mbar_init(&x.p_full, 4);
+        mbar_init(&x.p_empty[0], 1);
+        mbar_init(&x.p_empty[1], 1);
         mbar_init(&x.drain, 1);
         x.abort = 0;
         fence_mbar_init();
@@ -218,15 +232,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_alloc(&x.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
-    if (tid < 128) x.m_s[tid >> 6][tid & 63] = -INFINITY;
-    for (int b = tid; b < min(cnt, ROWS_SMEM); b += ATTN_THREADS) {
-        int first;
-        x.rows[b] = static_cast<uint8_t>(block_rows(a, __ldg(lst + b), bh, &first));
-    }
-    // V slots are read in full by the PV MMA (M = 128 head-dim rows, K = 128
-    // KV rows) even where a tile loads fewer rows; they start at zero so those
-    // rows are finite (P is zero there). Q rows past a partial query block
-    // only feed discarded output columns; zero them as well.
+    // The producers and the softmax read the list once per block; keep it on chip.
+    for (int b = tid; b < min(cnt, LIST_SMEM); b += ATTN_THREADS) x.lst[b] = __ldg(lst + b);
+    // V slots are read in full by the PV MMA (M = 128 head-dim rows); the
+    // second panel of a head_dim-64 slot is never loaded and must stay zero,
+    // and rows past a partial block must be finite (P is zero there). Q rows
+    // past a partial query block only feed discarded output columns.
     {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
         uint4* vz = reinterpret_cast<uint4*>(smem + L::OFF_V);
@@ -243,104 +254,145 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = x.tmem_base;
     volatile int* abort_flag = &x.abort;
 
-    if (warp == W_KPROD || warp == W_VPROD) {
-        // ------------------------------------------------------------ producers
-        if (lane == 0) {
-            const bool is_k = warp == W_KPROD;
-            const int nslots = is_k ? KSLOTS : VSLOTS;
-            uint64_t* full = is_k ? x.k_full : x.v_full;
-            uint64_t* empty = is_k ? x.k_empty : x.v_empty;
-            uint8_t* base = smem + (is_k ? L::OFF_K : L::OFF_V);
-            const uint32_t slot_bytes = is_k ? L::K_SLOT : L::V_SLOT;
-            const CUtensorMap* mfull = is_k ? &tm_k : &tm_v;
-            const CUtensorMap* mpart = is_k ? &tm_k_rem : &tm_v_rem;
-            tma_prefetch_desc(mfull);
-            if (is_k) {
-                const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
-                mbar_arrive_expect_tx(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
-                for (int p = 0; p < L::NP; ++p)
-                    tma_load_2d(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
-            }
-            int armed = 0;  // tiles whose loads were issued
-            for (int i = 0; i < n_tiles; ++i) {
-                const int nb = min(2, cnt - 2 * i);
+    if (warp == W_KPROD) {
+        // ------------------------------------------------------------ K (+ Q) producer (whole warp)
+        {
+            if (lane == 0) tma_prefetch_desc(&tm_k);
+            __syncwarp();
+            const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
+            mbar_arrive_expect_tx_elect(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
+            for (int p = 0; p < L::NP; ++p)
+                tma_load_2d_elect(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
+            int armed = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int nb = min(2, cnt - 2 * t);
                 int rows[2] = {0, 0}, first[2] = {0, 0};
                 for (int h = 0; h < nb; ++h) {
-                    const int g = __ldg(lst + 2 * i + h);
-                    rows[h] = block_rows(a, g, bh, &first[h]);
-                    if (rows[h] == 0 && is_k) record_error(a.err, DEVERR_LIST | 2);
+                    rows[h] = block_rows(a, list_entry(x.lst, lst, 2 * t + h), bh, &first[h]);
+                    if (rows[h] == 0 && lane == 0) record_error(a.err, DEVERR_LIST | 2);
                 }
                 const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NP);
-                const int s = i % nslots;
-                if (!mbar_wait(&empty[s], ((i / nslots) & 1) ^ 1, abort_flag, a.err, is_k ? 0x10 : 0x11)) break;
-                if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
-                else mbar_arrive(&full[s]);
+                const int s = t % KSLOTS;
+                if (!mbar_wait(&x.k_empty[s], ((t / KSLOTS) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
+                if (bytes) mbar_arrive_expect_tx_elect(&x.k_full[s], bytes);
+                else mbar_arrive_elect(&x.k_full[s]);
+                uint8_t* slot = smem + L::OFF_K + s * L::K_SLOT;
                 for (int h = 0; h < nb; ++h)
-                    if (rows[h]) load_block<D, IL>(base + s * slot_bytes, h, rows[h], first[h], mfull, mpart, &full[s]);
-                armed = i + 1;
+                    if (rows[h])
+                        load_block<D, IL>(slot + h * (IL ? L::BLOCK_IL : 64u * 128u), 128u * 128u, rows[h], first[h],
+                                          &tm_k, &tm_k_rem, &x.k_full[s]);
+                armed = t + 1;
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA exits.
-                if (is_k) mbar_drain(&x.q_full, 0, 10000000ull);
-                for (int i = max(0, armed - nslots); i < armed; ++i)
-                    mbar_drain(&full[i % nslots], (i / nslots) & 1, 10000000ull);
+                mbar_drain(&x.q_full, 0, 10000000ull);
+                for (int t = max(0, armed - KSLOTS); t < armed; ++t)
+                    mbar_drain(&x.k_full[t % KSLOTS], (t / KSLOTS) & 1, 10000000ull);
             }
         }
+    } else if (warp == W_VPROD) {
+        // ------------------------------------------------------------ V producer (whole warp)
+        {
+            if (lane == 0) tma_prefetch_desc(&tm_v);
+            __syncwarp();
+            int armed = 0;
+            for (int b = 0; b < cnt; ++b) {
+                int first = 0;
+                const int rows = block_rows(a, list_entry(x.lst, lst, b), bh, &first);
+                const int s = b % VSLOTS;
+                if (!mbar_wait(&x.v_empty[s], ((b / VSLOTS) & 1) ^ 1, abort_flag, a.err, 0x11)) break;
+                if (rows) {
+                    mbar_arrive_expect_tx_elect(&x.v_full[s], static_cast<uint32_t>(rows * 128 * L::NP));
+                    load_block<D, IL>(smem + L::OFF_V + s * L::V_SLOT, 64u * 128u, rows, first, &tm_v, &tm_v_rem,
+                                      &x.v_full[s]);
+                } else {
+                    mbar_arrive_elect(&x.v_full[s]);
+                }
+                armed = b + 1;
+            }
+            if (*abort_flag)
+                for (int b = max(0, armed - VSLOTS); b < armed; ++b)
+                    mbar_drain(&x.v_full[b % VSLOTS], (b / VSLOTS) & 1, 10000000ull);
+        }
     } else if (warp == W_MMA) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, true);
+        // ------------------------------------------------------------ MMA issuer (whole warp,
+        // one elected lane issues; every branch below is warp-uniform)
+        {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, false);
             const uint32_t sQ = smem_u32(smem + L::OFF_Q);
             const uint32_t sK = smem_u32(smem + L::OFF_K);
             const uint32_t sV = smem_u32(smem + L::OFF_V);
             const uint32_t sP = smem_u32(smem + L::OFF_P);
             bool issued_any = false;
             bool ok = mbar_wait(&x.q_full, 0, abort_flag, a.err, 0x20);
-            int next_s = 0, next_pv = 0;
+            int s_next = 0, s_half = 0;   // next S tile: step s_next, half s_half
+            int pv_next = 0, pv_blk = 0;  // next PV block: step pv_next, block pv_blk of 4
             unsigned long long stall_t0 = 0;
             uint32_t idle = 0;
-            while (ok && next_pv < n_tiles) {
+            while (ok && pv_next < n_steps) {
                 bool progressed = false;
-                // PV for the oldest tile whose P and V are ready (frees a V slot and a P buffer).
-                if (next_pv < next_s) {
-                    const int i = next_pv, g = i & 1, vs = i % VSLOTS;
-                    if (mbar_test(&x.p_full[g], (i >> 1) & 1) && mbar_test(&x.v_full[vs], (i / VSLOTS) & 1)) {
-                        tc_fence_after();
+                // PV blocks of the oldest step whose P is written (frees V slots and, at the
+                // end of the step, the P buffer).
+                if (pv_next < s_next && mbar_test(&x.p_full, pv_next & 1)) {
+                    const int g = pv_next & 1;
+                    while (pv_blk < 4) {
+                        const int b = 4 * pv_next + pv_blk;
+                        if (b < cnt) {
+                            const int vs = b % VSLOTS;
+                            if (!mbar_test(&x.v_full[vs], (b / VSLOTS) & 1)) break;
+                            tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            // A = V^T (M = head_dim, MN-major: 64-wide panels LBO apart, 8-row K groups SBO apart)
-                            const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + kk * L::KV_K16, L::KV_PANEL, L::KV_SBO);
-                            // B = P^T (N = 64 queries, MN-major, one 64-wide panel)
-                            const uint64_t bd = sdesc_sw128(sP + g * L::P_BUF + kk * 2048, L::P_BUF, 1024);
-                            umma_bf16(tmem + 256u + 64u * g, ad, bd, IDESC_O, (i >= 2 || kk > 0) ? 1u : 0u);
+                            for (int k4 = 0; k4 < 4; ++k4) {
+                                // A = V_block^T (M = head_dim, MN-major), B = P^T (N = 64 queries, K-major)
+                                const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + k4 * L::V_K16, L::V_LBO, L::V_SBO);
+                                const uint64_t bd = sdesc_sw128(sP + pv_blk * L::P_PANEL + k4 * 32, 16, 1024);
+                                umma_bf16_elect(tmem + TM_O + 64u * g, ad, bd, IDESC_O,
+                                          (pv_next >= 2 || pv_blk > 0 || k4 > 0) ? 1u : 0u);
+                            }
+                            umma_commit_elect(&x.v_empty[vs]);
+                            issued_any = true;
                         }
-                        umma_commit(&x.v_empty[vs]);
-                        umma_commit(&x.p_empty[g]);
-                        issued_any = true;
-                        ++next_pv;
+                        ++pv_blk;
                         progressed = true;
                     }
+                    if (pv_blk == 4) {
+                        umma_commit_elect(&x.p_empty[pv_next & 1]);
+                        ++pv_next;
+                        pv_blk = 0;
+                    }
                 }
-                // S for the next tile once its TMEM buffer is free and its K has landed.
-                if (next_s < n_tiles) {
-                    const int i = next_s, b = i & 3, ks = i % KSLOTS;
-                    const bool buf_free = i < 4 || mbar_test(&x.s_free[b], ((i >> 2) - 1) & 1);
-                    if (buf_free && mbar_test(&x.k_full[ks], (i / KSLOTS) & 1)) {
+                // S tiles: step s_next needs its TMEM buffer free and its K tile landed.
+                // S runs at most two steps ahead of the oldest PV not yet issued, so that
+                // a PV whose P is written does not queue behind more S work.
+                if (s_next < n_steps && s_next <= pv_next + 2) {
+                    const int bsel = s_next % SBUFS;
+                    const int t = 2 * s_next + s_half;
+                    const bool buf_free =
+                        s_half == 1 || s_next < SBUFS || mbar_test(&x.s_free[bsel], ((s_next / SBUFS) - 1) & 1);
+                    // (t < n_tiles always: a step with an empty second half ends after its first)
+                    if (buf_free && mbar_test(&x.k_full[t % KSLOTS], (t / KSLOTS) & 1)) {
                         tc_fence_after();
+                        const uint32_t ks = static_cast<uint32_t>(t % KSLOTS);
+                        const uint32_t d_addr = tmem + 128u * bsel + (s_half ? (16u << 16) : 0u);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t panel = static_cast<uint32_t>(kk >> 2);
-                            // A = K tile (M = 128 KV rows, K-major), B = Q (N = 64 queries, K-major)
-                            const uint64_t ad =
-                                sdesc_sw128(sK + ks * L::K_SLOT + panel * L::KV_PANEL + (kk & 3) * 32, 16, L::KV_SBO);
-                            const uint64_t bd = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
-                            umma_bf16(tmem + 64u * b, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                            // A = Q (M = 64 queries, K-major), B = K tile (N = 128 keys, K-major)
+                            const uint64_t ad = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd =
+                                sdesc_sw128(sK + ks * L::K_SLOT + panel * L::K_PANEL + (kk & 3) * 32, 16, L::K_SBO);
+                            umma_bf16_elect(d_addr, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
                         }
-                        umma_commit(&x.k_empty[ks]);
-                        umma_commit(&x.s_full[b]);
+                        umma_commit_elect(&x.k_empty[ks]);
                         issued_any = true;
-                        ++next_s;
+                        if (s_half == 1 || t + 1 >= n_tiles) {
+                            umma_commit_elect(&x.s_full[bsel]);
+                            ++s_next;
+                            s_half = 0;
+                        } else {
+                            s_half = 1;
+                        }
                         progressed = true;
                     }
                 }
@@ -358,187 +410,149 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
             if (*abort_flag && issued_any) {
-                umma_commit(&x.drain);
+                umma_commit_elect(&x.drain);
                 mbar_drain(&x.drain, 0, 10000000ull);
             }
         }
     } else if (warp >= W_SOFT0) {
         // ------------------------------------------------------------ softmax
-        const int g = (warp - W_SOFT0) >> 2;   // this warpgroup takes the tiles i with i % 2 == g
+        const int g = (warp - W_SOFT0) >> 2;   // this warpgroup takes the steps s with s % 2 == g
         const int sp = warp & 3;               // TMEM sub-partition of this warp
-        const int t = sp * 32 + lane;          // KV token of a tile / head-dim row of O^T
+        const int qr = sp * 16 + (lane & 15);  // query row of this thread's S lane
+        const int hh = lane >> 4;              // which tile of the step
         const int bar_id = 1 + g;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
-        const uint32_t o_col = 256u + 64u * static_cast<uint32_t>(g);
+        const uint32_t o_col = TM_O + 64u * static_cast<uint32_t>(g);
         const float sl2 = a.scale_log2;
-        uint8_t* pbuf = smem + L::OFF_P + g * L::P_BUF + (t >> 3) * 1024 + (t & 7) * 128;
-        float l[64];  // this thread's share of each column's softmax denominator
-#pragma unroll
-        for (int c = 0; c < 64; ++c) l[c] = 0.f;
+        // this thread's P row: panels 2*hh and 2*hh+1 (keys 128*hh ... 128*hh+127 of the step)
+        uint8_t* prow = smem + L::OFF_P + (2 * hh) * L::P_PANEL + qr * 128;
+        float m_run = -INFINITY;  // stabiliser of this row (identical in lanes l and l^16)
+        float l_run = 0.f;        // this thread's share of the row's softmax denominator
 
-        for (int i = g; i < n_tiles; i += 2) {
-            const int j = i >> 1;  // local tile index of this warpgroup
-            const int bi = 2 * i + (t >> 6);
-            int rows = 0;
-            if (bi < cnt) {
-                if (bi < ROWS_SMEM) {
-                    rows = x.rows[bi];
-                } else {
-                    int first;
-                    rows = block_rows(a, __ldg(lst + bi), bh, &first);
-                }
-            }
-            const bool valid = (t & 63) < rows;
-            const uint32_t s_addr = lane_base + 64u * static_cast<uint32_t>(i & 3);
-            mbar_wait(&x.s_full[i & 3], (i >> 2) & 1, abort_flag, a.err, 0x30);
+        int j = 0;  // local step index of this warpgroup
+        for (int s = g; s < n_steps; s += 2, ++j) {
+            const int tile = 2 * s + hh;
+            const int rows0 = entry_rows(a, x.lst, lst, 2 * tile, cnt);
+            const int rows1 = entry_rows(a, x.lst, lst, 2 * tile + 1, cnt);
+            const int bsel = s % SBUFS;
+            mbar_wait(&x.s_full[bsel], (s / SBUFS) & 1, abort_flag, a.err, 0x30);
             __syncwarp();
             tc_fence_after();
-            // 1. Does any score exceed the stabiliser by more than the lazy bound?
-            float xmax = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float s[32];
-                tmem_ld32(s_addr + 32u * h, s);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(&x.m_s[g][32 * h + c]);
-                    s[c] = fmaf(s[c], sl2, -m4.x);
-                    s[c + 1] = fmaf(s[c + 1], sl2, -m4.y);
-                    s[c + 2] = fmaf(s[c + 2], sl2, -m4.z);
-                    s[c + 3] = fmaf(s[c + 3], sl2, -m4.w);
-                }
-#pragma unroll
-                for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                    for (int c = 0; c < w; ++c) s[c] = fmaxf(s[c], s[c + w]);
-                xmax = fmaxf(xmax, s[0]);
-            }
-            if (!valid) xmax = -INFINITY;
-            const bool need = named_bar_or(bar_id, 128, xmax > LAZY_RESCALE_LOG2);
-            // PV of this warpgroup's previous tile must be done before its P
-            // buffer is rewritten or its O^T columns are rescaled.
-            if (j > 0) mbar_wait(&x.p_empty[g], (j - 1) & 1, abort_flag, a.err, 0x31);
+            float sv[128];
+            tmem_ld128_nowait(lane_base + 128u * bsel, sv);
+            tmem_ld_wait();
+            tc_fence_before();
             __syncwarp();
-            if (need) {
-                // 2. Exact column maxima of this tile over its 128 KV tokens.
-                __syncwarp();
+            if (lane == 0) mbar_arrive(&x.s_free[bsel]);
+            // 1. Row maximum over the valid keys of the step (masked keys -> -inf).
+            if (!__all_sync(0xffffffffu, rows0 == 64 && rows1 == 64)) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float s[32];
-                    tmem_ld32(s_addr + 32u * h, s);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) s[c] = valid ? s[c] * sl2 : -INFINITY;
-                    transpose_reduce<true>(s, lane);
-                    x.red[g][sp][32 * h + lane] = s[0];
+                for (int c = 0; c < 128; ++c) {
+                    const bool ok = c < 64 ? (c < rows0) : (c - 64 < rows1);
+                    sv[c] = ok ? sv[c] : -INFINITY;
                 }
+            }
+            float mx;
+            {
+                float m3[43];
+#pragma unroll
+                for (int i = 0; i < 42; ++i) m3[i] = fmax3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
+                m3[42] = fmaxf(sv[126], sv[127]);
+                float m2[15];
+#pragma unroll
+                for (int i = 0; i < 14; ++i) m2[i] = fmax3(m3[3 * i], m3[3 * i + 1], m3[3 * i + 2]);
+                m2[14] = m3[42];
+                float m1[5];
+#pragma unroll
+                for (int i = 0; i < 5; ++i) m1[i] = fmax3(m2[3 * i], m2[3 * i + 1], m2[3 * i + 2]);
+                mx = fmaxf(fmax3(m1[0], m1[1], m1[2]), fmaxf(m1[3], m1[4]));
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float ms = mx * sl2;
+            const bool need = ms > m_run + LAZY_RESCALE_LOG2;
+            const float m_new = need ? ms : m_run;
+            const float alpha = need ? fast_exp2(m_run - m_new) : 1.f;  // 0 when m_run = -inf
+            l_run *= alpha;
+            m_run = m_new;
+            // 2. Probabilities (registers), then wait until PV of the previous step
+            // has read the P buffer (it also ends this warpgroup's last PV).
+            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+            uint32_t pk[64];
+            float la = 0.f, lb = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; c += 2) {
+                float e0, e1;
+                ffma2_bc(e0, e1, sv[c], sv[c + 1], sl2, -mu);
+                const float p0 = fast_exp2(e0);
+                const float p1 = fast_exp2(e1);
+                fadd2_acc(la, lb, p0, p1);
+                pk[c >> 1] = pack_bf16x2(p0, p1);
+            }
+            l_run += la + lb;
+            if (s > 0) mbar_wait(&x.p_empty[(s - 1) & 1], ((s - 1) >> 1) & 1, abort_flag, a.err, 0x31);
+            // 3. P row -> shared memory (two 64-key panels, 128-byte swizzle).
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int chunk = c ^ (qr & 7);
+                    const int k = 32 * pp + 4 * c;
+                    *reinterpret_cast<uint4*>(prow + pp * L::P_PANEL + chunk * 16) =
+                        make_uint4(pk[k], pk[k + 1], pk[k + 2], pk[k + 3]);
+                }
+            }
+            // 4. Rescale O^T columns of rows whose stabiliser moved (rare after the
+            // first steps); the previous PV into O^T has completed (waited above).
+            if (j > 0 && named_bar_or(bar_id, 128, need)) {
+                if (hh == 0) x.alpha[g][qr] = alpha;
                 named_bar_sync(bar_id, 128);
-                float alpha[2], m_new[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = 32 * h + lane;  // lane owns column c of this half
-                    const float m_old = x.m_s[g][c];
-                    m_new[h] = fmaxf(m_old, fmaxf(fmaxf(x.red[g][0][c], x.red[g][1][c]),
-                                                  fmaxf(x.red[g][2][c], x.red[g][3][c])));
-                    alpha[h] = (m_new[h] == -INFINITY) ? 1.f : fast_exp2(m_old - m_new[h]);
-                }
-                named_bar_sync(bar_id, 128);  // every warp has read the old maxima
-                if (sp == 0) {
-                    x.m_s[g][lane] = m_new[0];
-                    x.m_s[g][32 + lane] = m_new[1];
-                }
                 tc_fence_after();
                 __syncwarp();
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if (j > 0) {
-                        float o[32];
-                        tmem_ld32(lane_base + o_col + 32u * h, o);
-                        tmem_ld_wait();
+                    float o[32];
+                    tmem_ld32(lane_base + o_col + 32u * h, o);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] *= __shfl_sync(0xffffffffu, alpha[h], c);
-                        tmem_st32(lane_base + o_col + 32u * h, o);
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(&x.alpha[g][32 * h + c]);
+                        o[c] *= a4.x;
+                        o[c + 1] *= a4.y;
+                        o[c + 2] *= a4.z;
+                        o[c + 3] *= a4.w;
                     }
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) l[32 * h + c] *= __shfl_sync(0xffffffffu, alpha[h], c);
+                    tmem_st32(lane_base + o_col + 32u * h, o);
                 }
-                if (j > 0) tmem_st_wait();
-                named_bar_sync(bar_id, 128);
-            }
-            // 3. Probabilities P = 2^(s*scale*log2e - m) as bf16 P^T rows.
-            __syncwarp();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float s[32];
-                tmem_ld32(s_addr + 32u * h, s);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(&x.m_s[g][32 * h + c]);
-                    const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; e += 2) {
-                        const float p0 = valid ? fast_exp2(fmaf(s[c + e], sl2, -mm[e])) : 0.f;
-                        const float p1 = valid ? fast_exp2(fmaf(s[c + e + 1], sl2, -mm[e + 1])) : 0.f;
-                        l[32 * h + c + e] += p0;
-                        l[32 * h + c + e + 1] += p1;
-                        pk[(c + e) >> 1] = pack_bf16x2(p0, p1);
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int chunk = (4 * h + k) ^ (t & 7);
-                    *reinterpret_cast<uint4*>(pbuf + chunk * 16) =
-                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-                }
+                tmem_st_wait();
+                named_bar_sync(bar_id, 128);  // alpha reads done before it is rewritten
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&x.s_free[i & 3]);
-                mbar_arrive(&x.p_full[g]);
-            }
+            if (lane == 0) mbar_arrive(&x.p_full);
         }
 
         // ------------------------------------------------------------ epilogue
-        const int n_g = (n_tiles - g + 1) >> 1;  // tiles this warpgroup took
-        if (n_g > 0) mbar_wait(&x.p_empty[g], (n_g - 1) & 1, abort_flag, a.err, 0x34);
-        __syncwarp();
-        tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float v[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = l[32 * h + c];
-            transpose_reduce<false>(v, lane);
-            x.red[g][sp][32 * h + lane] = v[0];
+        const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+        if (hh == 0) {
+            x.lsum[g][qr] = l_row;
+            x.m_s[g][qr] = m_run;
         }
-        named_bar_sync(bar_id, 128);
-        if (sp == 0) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = 32 * h + lane;
-                x.lsum[g][c] = x.red[g][0][c] + x.red[g][1][c] + x.red[g][2][c] + x.red[g][3][c];
-            }
-        }
+        // the last PV of the call ends every PV of both warpgroups
+        if (n_steps > 0)
+            mbar_wait(&x.p_empty[(n_steps - 1) & 1], ((n_steps - 1) >> 1) & 1, abort_flag, a.err, 0x34);
         tc_fence_before();
         named_bar_sync(3, 256);  // both warpgroups: sums, maxima and last PVs are final
         tc_fence_after();
         // Warpgroup g merges and writes query columns [32g, 32g + 32).
-        const int n0 = (n_tiles + 1) >> 1, n1 = n_tiles >> 1;
+        const int n0 = (n_steps + 1) >> 1, n1 = n_steps >> 1;
         float o0[32], o1[32];
         __syncwarp();
-        if (n0 > 0) {
-            tmem_ld32(lane_base + 256u + 32u * g, o0);
-        }
-        if (n1 > 0) {
-            tmem_ld32(lane_base + 320u + 32u * g, o1);
-        }
+        tmem_ld32(lane_base + TM_O + 32u * g, o0);
+        tmem_ld32(lane_base + TM_O + 64u + 32u * g, o1);
         tmem_ld_wait();
         __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K);
+        const int t = sp * 32 + lane;
         if (t < D) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
