@@ -4,12 +4,14 @@
 // Technical Summary 2.2 "Token Compression").
 //
 // HBM-bound. One CTA per (batch*head, frame): K frames first, then the query
-// frames of the current chunk. A frame is streamed block by block (64 tokens x
-// head_dim bf16, contiguous) with 128-bit coalesced loads, UNROLL blocks in
-// flight per thread. Each block's column sums are reduced with warp shuffles
-// inside a warp and then across the CTA's 8 warps in a fixed order through
-// shared memory (deterministic). The frame mean is the sum of the frame's block
-// sums divided by the frame's token count, so K is read once.
+// frames of the current chunk. Warp w of the CTA owns blocks w, w+8, w+16, ...
+// of its frame and streams each block (64 tokens x head_dim bf16, 16 KB,
+// contiguous) with 128-bit coalesced loads, 16 per lane in flight; a block's
+// column sums are reduced with warp shuffles only, so no CTA-wide barrier sits
+// between loads and 64 KB per CTA stay in flight. The frame sum is each warp's
+// running sum of its block sums, combined across the 8 warps in a fixed order
+// through shared memory once at the end (deterministic), then divided by the
+// frame's token count, so K is read once.
 #include "lf_internal.h"
 
 #include <cuda_bf16.h>
@@ -40,18 +42,16 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& u)
     }
 }
 
-template <int D, int UNROLL>
-__global__ void __launch_bounds__(POOL_THREADS) pool_kernel(const PoolArgs a)
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
 {
-    constexpr int CPR = D / 8;                              // 16-byte chunks per token row
-    constexpr int RPI = 32 / CPR;                           // rows one warp load covers
-    constexpr int ROWS_PER_WARP = BLOCK_TOKENS / POOL_WARPS;  // 8 rows of a block per warp
-    constexpr int LOADS = ROWS_PER_WARP / RPI;              // loads per lane per block
-    static_assert(LOADS >= 1 && ROWS_PER_WARP % RPI == 0, "layout");
-    static_assert(UNROLL * D <= POOL_THREADS, "final reduction needs UNROLL*D threads");
+    constexpr int CPR = D / 8;          // 16-byte chunks per token row
+    constexpr int RPL = 32 / CPR;       // rows one warp-wide load covers
+    constexpr int LOADS = BLOCK_TOKENS / RPL;  // loads per lane per block
+    constexpr int PHASE = 16;           // loads in flight per lane
+    static_assert(LOADS % PHASE == 0, "layout");
 
-    __shared__ float red[UNROLL][POOL_WARPS][D];
-    __shared__ float bsum[UNROLL][D];
+    __shared__ float red[POOL_WARPS][D];
 
     const int units = a.NF + a.n_cur;
     const int bh = blockIdx.x / units;
@@ -70,58 +70,48 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(const PoolArgs a)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunk = lane % CPR, rsub = lane / CPR;
-    float frame_acc = 0.f;
+    float facc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // this warp's share of the frame sum
 
-    for (int j0 = 0; j0 < a.bpf; j0 += UNROLL) {
-        uint4 buf[UNROLL][LOADS];
+    for (int j = warp; j < a.bpf; j += POOL_WARPS) {
+        const int nrows = min(BLOCK_TOKENS, a.F - j * BLOCK_TOKENS);
+        const uint16_t* bsrc = src + static_cast<long long>(j) * BLOCK_TOKENS * D + chunk * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int j = j0 + u;
-            const int nrows = (j < a.bpf) ? min(BLOCK_TOKENS, a.F - j * BLOCK_TOKENS) : 0;
+        for (int ph = 0; ph < LOADS / PHASE; ++ph) {
+            uint4 buf[PHASE];
 #pragma unroll
-            for (int l = 0; l < LOADS; ++l) {
-                const int row = warp * ROWS_PER_WARP + l * RPI + rsub;
-                if (row < nrows)
-                    buf[u][l] = ld_stream_v4(src + static_cast<long long>(j * BLOCK_TOKENS + row) * D + chunk * 8);
-                else
-                    buf[u][l] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < PHASE; ++i) {
+                const int row = (ph * PHASE + i) * RPL + rsub;
+                buf[i] = row < nrows ? ld_stream_v4(bsrc + static_cast<long long>(row) * D) : make_uint4(0u, 0u, 0u, 0u);
             }
+#pragma unroll
+            for (int i = 0; i < PHASE; ++i) add_bf16x8(acc, buf[i]);
         }
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int off = CPR; off < 32; off <<= 1)
 #pragma unroll
-            for (int l = 0; l < LOADS; ++l) add_bf16x8(acc, buf[u][l]);
+            for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+        if (rsub == 0) {
+            float4* o = reinterpret_cast<float4*>(dst + static_cast<long long>(j) * D + chunk * 8);
+            const float n = static_cast<float>(nrows);
+            o[0] = make_float4(acc[0] / n, acc[1] / n, acc[2] / n, acc[3] / n);
+            o[1] = make_float4(acc[4] / n, acc[5] / n, acc[6] / n, acc[7] / n);
 #pragma unroll
-            for (int off = CPR; off < 32; off <<= 1)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-            if (rsub == 0) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) red[u][warp][chunk * 8 + i] = acc[i];
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x < UNROLL * D) {
-            const int u = threadIdx.x / D, col = threadIdx.x - u * D;
-            const int j = j0 + u;
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < POOL_WARPS; ++w) s += red[u][w][col];
-            if (j < a.bpf) {
-                const int nrows = min(BLOCK_TOKENS, a.F - j * BLOCK_TOKENS);
-                dst[static_cast<long long>(j) * D + col] = s / static_cast<float>(nrows);
-            }
-            bsum[u][col] = (j < a.bpf) ? s : 0.f;
-        }
-        __syncthreads();
-        if (is_k && threadIdx.x < D) {
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) frame_acc += bsum[u][threadIdx.x];
+            for (int i = 0; i < 8; ++i) facc[i] += acc[i];
         }
     }
-    if (is_k && threadIdx.x < D)
-        a.k_frame[(static_cast<long long>(bh) * a.NF + f) * D + threadIdx.x] = frame_acc / static_cast<float>(a.F);
+    if (!is_k) return;
+    if (rsub == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp][chunk * 8 + i] = facc[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < POOL_WARPS; ++w) s += red[w][threadIdx.x];
+        a.k_frame[(static_cast<long long>(bh) * a.NF + f) * D + threadIdx.x] = s / static_cast<float>(a.F);
+    }
 }
 
 }  // namespace
@@ -131,9 +121,9 @@ cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s)
     const long long grid = static_cast<long long>(a.BH) * (a.NF + a.n_cur);
     if (grid <= 0) return cudaSuccess;
     if (a.D == 128)
-        pool_kernel<128, 2><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
+        pool_kernel<128><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
     else
-        pool_kernel<64, 4><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
+        pool_kernel<64><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
     return cudaGetLastError();
 }
 
