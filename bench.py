@@ -47,6 +47,9 @@ def _args():
     p.add_argument("--workload", default="layer480p")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the per-config report (all five workloads, rollout per chunk)")
+    p.add_argument("--config-steps", type=int, default=30)
     return p.parse_args()
 
 
@@ -268,6 +271,108 @@ def _attn_traffic():
     return d.get("dram_bytes_per_launch") if d.get("kernel_src_sha256") == sha else None
 
 
+def _pct(xs, p):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, max(0, int(round(p / 100.0 * (len(xs) - 1)))))]
+
+
+def measure_call(L, shape, chunk_index, topk_frames, kb, q, k, v, steps, warmup, flush):
+    """Time the four calls of one HSA call on resident inputs (L2 flushed before
+    every step); returns µs per kernel (mean, p10, p90), credited FLOPs and
+    pooling bytes."""
+    import torch
+    call = L.HSACall(shape, chunk_index, topk_frames, kb)
+    b = call.buf
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, warmup)):
+        call(q, k, v)
+    torch.cuda.synchronize()
+    flops = credited_flops(b.block_list.cpu().numpy(), b.block_count.cpu().numpy(),
+                           shape.frame_tokens, shape.bpf, shape.head_dim, shape.n_cur)
+    E = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        e = E[i]
+        e[0].record(stream)
+        call.pool(q, k)
+        e[1].record(stream)
+        L.lf_select_frames(shape, chunk_index, topk_frames, b.q_pool, b.k_frame, b.frame_sel)
+        e[2].record(stream)
+        L.lf_select_blocks(shape, chunk_index, topk_frames, kb, b.q_pool, b.k_pool, b.frame_sel,
+                           b.block_list, b.block_count, b.list_cap)
+        e[3].record(stream)
+        call.attend(q, k, v)
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    st, detail = L.lf_get_device_error()
+    if st != 0:
+        raise SystemExit(f"device error: {st} {detail:#x}")
+
+    def us(i0, i1):
+        xs = [E[j][i0].elapsed_time(E[j][i1]) * 1e3 for j in range(steps)]
+        return statistics.mean(xs), _pct(xs, 10), _pct(xs, 90)
+
+    pool_bytes = (q.numel() + k.numel()) * 2 + (b.q_pool.numel() + b.k_pool.numel() + b.k_frame.numel()) * 4
+    return dict(pool=us(0, 1), select_frames=us(1, 2), select_blocks=us(2, 3), attn=us(3, 4),
+                total=us(0, 4), flops=flops, pool_bytes=pool_bytes, kb=kb,
+                list_entries=int(b.block_count.sum().item()))
+
+
+def _summary(m, peaks):
+    t = m["total"][0]
+    att = m["attn"][0]
+    return {
+        "us_per_call": round(t, 2), "us_p10_p90": [round(m["total"][1], 2), round(m["total"][2], 2)],
+        "kernels_us": {k: round(m[k][0], 2) for k in ("pool", "select_frames", "select_blocks", "attn")},
+        "kept_tflop": round(m["flops"] / 1e12, 5), "topk_blocks": m["kb"],
+        "tflops_call": round(m["flops"] / (t * 1e-6) / 1e12, 1),
+        "attn_tflops": round(m["flops"] / (att * 1e-6) / 1e12, 1),
+        "attn_frac_of_bf16_peak": round(m["flops"] / (att * 1e-6) / 1e12 / peaks["bf16"], 4),
+        "pool_frac_of_hbm": round(m["pool_bytes"] / (m["pool"][0] * 1e-6) / 1e9 / peaks["hbm"], 3),
+        "select_over_attn": round((m["pool"][0] + m["select_frames"][0] + m["select_blocks"][0]) / att, 4),
+    }
+
+
+def config_report(L, lf_synth, peaks, steps, flush):
+    """The other workloads of the benchmark plan at one GPU: tiny, long-video,
+    pattern-diversity batch at two sparsities, and the 7-chunk rollout with the
+    Chunk-Aware Growth budgets (per chunk and the total)."""
+    import torch
+    out = {}
+    for name, kbs in (("tiny", [None]), ("longvideo480p", [None]), ("patterns480p", [12, 6])):
+        w = lf_synth.CONFIGS[name]
+        shape = L.shape_from_workload(w)
+        q, k, v = (t.cuda() for t in lf_synth.make_qkv(w))
+        for kb in kbs:
+            kbv = kb or _kb(L, shape, w)
+            m = measure_call(L, shape, w.chunk_index, w.topk_frames, kbv, q, k, v, steps, 3, flush)
+            out[name if kb is None else f"{name}_kb{kb}"] = _summary(m, peaks)
+        del q, k, v
+        torch.cuda.empty_cache()
+    w = lf_synth.CONFIGS["rollout480p"]
+    qa, ka, va = lf_synth.make_rollout_qkv(w)
+    n = int(w.extra["n_chunks"])
+    st, s_out, beta = L.lf_cag_budget(list(range(1, n + 1)), list(range(1, n + 1)), w.extra["s_base"], w.sparsity)
+    if st != 0:
+        raise SystemExit(f"CAG budgets infeasible: status {st}")
+    chunks, tot_us, tot_flops = [], 0.0, 0.0
+    for c in range(1, n + 1):
+        wc, q, k, v = lf_synth.rollout_chunk(w, qa, ka, va, c)
+        shape = L.shape_from_workload(wc)
+        n_sel = L.lf_frames_selected(shape, c, wc.topk_frames)
+        kb = shape.bpf if c == 1 else L.lf_blocks_for_sparsity(s_out[c - 1], shape.Nkv, n_sel, shape.bpf)
+        q, k, v = q.cuda(), k.cuda(), v.cuda()
+        m = measure_call(L, shape, c, wc.topk_frames, kb, q, k, v, steps, 3, flush)
+        sm = _summary(m, peaks)
+        sm["chunk"], sm["s_i"] = c, round(float(s_out[c - 1]), 6)
+        chunks.append(sm)
+        tot_us += m["total"][0]
+        tot_flops += m["flops"]
+    out["rollout480p"] = {"beta": round(float(beta), 6), "chunks": chunks, "total_us": round(tot_us, 1),
+                          "tflops": round(tot_flops / (tot_us * 1e-6) / 1e12, 1)}
+    return out
+
+
 def run_ours(a):
     import numpy as np
     import torch
@@ -327,6 +432,15 @@ def run_ours(a):
         return statistics.mean(E[s][i0].elapsed_time(E[s][i1]) for s in range(a.steps))
 
     t_pool, t_sf, t_sb, t_attn = mean_ms(0, 1), mean_ms(1, 2), mean_ms(2, 3), mean_ms(3, 4)
+    step_ms = [E[s][0].elapsed_time(E[s][4]) for s in range(a.steps)]
+    # attention alone, back to back with a warm L2 (K/V of the call stay resident)
+    ew = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    for s0, s1 in ew:
+        s0.record(stream)
+        call.attend(q, k, v)
+        s1.record(stream)
+    torch.cuda.synchronize()
+    t_attn_warm = statistics.mean(s0.elapsed_time(s1) for s0, s1 in ew)
     t_step = mean_ms(0, 4)
     t_step_max = _max_over_ranks(dist, t_step)
     value = ws * flops / (t_step_max * 1e-3) / 1e12
@@ -363,6 +477,8 @@ def run_ours(a):
         "data": "synthetic (lf_synth, seeded; stands in for the pages' VBench 480p rollouts)",
         "config": _config(w, kb),
         "us_per_call": t_step_max * 1e3,
+        "us_p10_p90": [_pct(step_ms, 10) * 1e3, _pct(step_ms, 90) * 1e3],
+        "attn_us_warm_l2": t_attn_warm * 1e3,
         "kernels_us": {"pool": t_pool * 1e3, "select_frames": t_sf * 1e3,
                        "select_blocks": t_sb * 1e3, "block_sparse_attn": t_attn * 1e3},
         "kept_tflop_per_call": flops / 1e12,
@@ -382,6 +498,8 @@ def run_ours(a):
         "clocks": clk.summary(),
         "wall_s_timed_region": wall,
     }
+    if rank == 0 and not a.no_configs:
+        line["configs"] = config_report(L, lf_synth, peaks, a.config_steps, flush)
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         r = _oracle_sample(w, a.cpu_budget_s, q_h, k_h, v_h)
         line["cpu_baseline"] = {"value": r["flops"] / r["t_call"] / 1e12, "unit": "TFLOP/s",
