@@ -152,11 +152,14 @@ class ClockSampler:
 
 
 def _dist():
+    """(dist module or None, rank, world size, local rank). One process per GPU;
+    the process group (NCCL, or gloo when LF_DIST_BACKEND=gloo for host-only
+    tests) carries only the barrier and the max-over-ranks timing."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
         import torch.distributed as dist
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.init_process_group(os.environ.get("LF_DIST_BACKEND", "nccl"), timeout=timedelta(seconds=120))
         return dist, dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
     return None, 0, 1, 0
 
@@ -165,9 +168,18 @@ def _max_over_ranks(dist, x):
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _rank_workload(name, rank):
+    """Weak scaling: every rank runs its own independent call of the same shape
+    (different (batch, head) data: the seed is offset by the rank)."""
+    import lf_synth
+    w = lf_synth.CONFIGS[name]
+    return w if rank == 0 else lf_synth.workload(name, seed=w.seed + 1000 * rank)
 
 
 def _oracle_sample(w, budget_s, q, k, v, block_list=None, block_count=None):
@@ -382,7 +394,7 @@ def run_ours(a):
     import block_sparse_attention_lf_b200 as L
     import lf_synth
 
-    w = _workload(a.workload)
+    w = _rank_workload(a.workload, rank)
     shape = L.shape_from_workload(w)
     kb = _kb(L, shape, w)
     q_h, k_h, v_h = lf_synth.make_qkv(w)
