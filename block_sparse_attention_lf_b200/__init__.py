@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblf_hsa.so")
 
 __all__ = [
-    "LfShape", "LfError", "lib", "lf_pool", "lf_select_frames", "lf_select_blocks",
+    "LfShape", "LfError", "lib", "lf_pool", "lf_pool_range", "lf_select_frames", "lf_select_blocks",
     "lf_block_sparse_attn", "lf_cag_budget", "lf_blocks_for_sparsity", "lf_frames_selected",
     "lf_list_capacity", "lf_get_device_error", "lf_status_string", "lf_version", "HSACall",
     "ABI_FUNCTIONS",
@@ -32,7 +32,7 @@ __all__ = [
 
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
-    "lf_pool", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
+    "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
     "lf_block_sparse_attn", "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error",
     "lf_status_string", "lf_version",
 )
@@ -98,6 +98,7 @@ def _load() -> ctypes.CDLL:
     S = ctypes.POINTER(LfShape)
     sig = {
         "lf_pool": ([S, P, P, P, P, P, P], I32),
+        "lf_pool_range": ([S, P, P, I32, I32, I32, P, P, P, P], I32),
         "lf_frames_selected": ([S, I32, I32], I32),
         "lf_select_frames": ([S, I32, I32, P, P, P, P], I32),
         "lf_list_capacity": ([S, I32, I32, I32], I32),
@@ -168,6 +169,19 @@ def lf_list_capacity(shape: LfShape, chunk_index: int, topk_frames: int, topk_bl
 
 def lf_blocks_for_sparsity(s: float, n_kv_blocks: int, n_sel_frames: int, bpf: int) -> int:
     return _lib.lf_blocks_for_sparsity(float(s), n_kv_blocks, n_sel_frames, bpf)
+
+
+def lf_pool_range(shape: LfShape, q, k, frame_begin: int, frame_end: int, q_pool, k_pool, k_frame,
+                  pool_q: bool = True, stream=None) -> None:
+    """Pool KV frames [frame_begin, frame_end) (and q when ``pool_q``) into the
+    same buffers lf_pool fills; other entries are left as they are."""
+    import torch
+    bf = _bf16()
+    qp = _dev_ptr(q, bf, "q") if pool_q else None
+    qpp = _dev_ptr(q_pool, torch.float32, "q_pool") if pool_q else None
+    _check(_lib.lf_pool_range(ctypes.byref(shape), qp, _dev_ptr(k, bf, "k"), int(frame_begin), int(frame_end),
+                              1 if pool_q else 0, qpp, _dev_ptr(k_pool, torch.float32, "k_pool"),
+                              _dev_ptr(k_frame, torch.float32, "k_frame"), _stream(stream)), "lf_pool_range")
 
 
 def lf_pool(shape: LfShape, q, k, q_pool, k_pool, k_frame, stream=None) -> None:

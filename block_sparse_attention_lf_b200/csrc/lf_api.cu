@@ -182,17 +182,27 @@ int32_t lf_list_capacity(const lf_hsa_shape* shape, int32_t chunk_index, int32_t
     return frames_selected(d, chunk_index, topk_frames) * blocks_per_frame(d, chunk_index, topk_blocks);
 }
 
-lf_status lf_pool(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, float* q_pool, float* k_pool,
-                  float* k_frame, void* stream)
+lf_status lf_pool_range(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, int32_t frame_begin,
+                        int32_t frame_end, int32_t pool_q, float* q_pool, float* k_pool, float* k_frame, void* stream)
 {
     Derived d;
     lf_status st = check_shape(shape, &d);
     if (st != LF_OK) return st;
-    if (!q || !k || !q_pool || !k_pool || !k_frame) return LF_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_frame))
+    if (frame_begin < 0 || frame_end < frame_begin || frame_end > d.NF) return LF_ERR_ARG;
+    if (!k || !k_pool || !k_frame || (pool_q && (!q || !q_pool))) return LF_ERR_NULL;
+    if (!aligned16(k) || !aligned16(k_pool) || !aligned16(k_frame) || (pool_q && (!aligned16(q) || !aligned16(q_pool))))
         return LF_ERR_ALIGN;
-    lf::PoolArgs a{q, k, q_pool, k_pool, k_frame, d.B * d.H, d.D, d.F, d.bpf, d.NF, d.n_cur, d.kv_stride};
+    lf::PoolArgs a{q, k, q_pool, k_pool, k_frame, d.B * d.H, d.D, d.F, d.bpf, d.NF, d.n_cur, d.kv_stride,
+                   frame_begin, frame_end - frame_begin, pool_q ? 1 : 0};
     return launch_status(lf::launch_pool(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_pool(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, float* q_pool, float* k_pool,
+                  float* k_frame, void* stream)
+{
+    if (!q || !q_pool) return LF_ERR_NULL;
+    const int32_t nf = shape ? shape->n_frames : 0;
+    return lf_pool_range(shape, q, k, 0, nf, 1, q_pool, k_pool, k_frame, stream);
 }
 
 lf_status lf_select_frames(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, const float* q_pool,

@@ -16,6 +16,8 @@ struct PoolArgs {
     float* k_frame;
     int BH, D, F, bpf, NF, n_cur;
     long long kv_stride;  // tokens between heads in k
+    int f0, nk;           // KV frames [f0, f0 + nk) are pooled
+    int pool_q;           // also pool the query frames
 };
 
 struct SelectFramesArgs {

@@ -3,8 +3,8 @@
 // pooling of q and k, frame-level compression of the keys; gist.science
 // Technical Summary 2.2 "Token Compression").
 //
-// HBM-bound. One CTA per (batch*head, frame): K frames first, then the query
-// frames of the current chunk. Warp w of the CTA owns blocks w, w+8, w+16, ...
+// HBM-bound. One CTA per (batch*head, frame): the pooled K frames first, then
+// the query frames of the current chunk. Warp w of the CTA owns blocks w, w+8, w+16, ...
 // of its frame and streams each block (64 tokens x head_dim bf16, 16 KB,
 // contiguous) with 128-bit coalesced loads, 16 per lane in flight; a block's
 // column sums are reduced with warp shuffles only, so no CTA-wide barrier sits
@@ -53,10 +53,11 @@ __global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
 
     __shared__ float red[POOL_WARPS][D];
 
-    const int units = a.NF + a.n_cur;
+    const int units = a.nk + (a.pool_q ? a.n_cur : 0);
     const int bh = blockIdx.x / units;
-    const int f = blockIdx.x - bh * units;
-    const bool is_k = f < a.NF;
+    const int u = blockIdx.x - bh * units;
+    const bool is_k = u < a.nk;
+    const int f = is_k ? a.f0 + u : a.NF + (u - a.nk);
     const uint16_t* src;
     float* dst;
     if (is_k) {
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
 
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s)
 {
-    const long long grid = static_cast<long long>(a.BH) * (a.NF + a.n_cur);
+    const long long grid = static_cast<long long>(a.BH) * (a.nk + (a.pool_q ? a.n_cur : 0));
     if (grid <= 0) return cudaSuccess;
     if (a.D == 128)
         pool_kernel<128><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);

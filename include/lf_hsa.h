@@ -9,6 +9,7 @@
  * Attention" (gist.science, Technical Summary 2.2):
  *
  *   lf_pool              block mean pooling of q and k, frame mean pooling of k
+ *   lf_pool_range        the same for a range of KV frames (pooled-key cache)
  *   lf_select_frames     per query block: frame scores, top-k memory frames T_r
  *                        plus the always-kept sink / recent / current frames
  *   lf_select_blocks     per selected frame: block scores, top-k blocks J_r(tau),
@@ -108,6 +109,25 @@ typedef struct lf_hsa_shape {
  */
 LF_API lf_status lf_pool(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
                   float* q_pool, float* k_pool, float* k_frame, void* stream);
+
+/*
+ * Token compression of a range of KV frames only: writes the k_pool rows and
+ * k_frame entries of frames [frame_begin, frame_end) (same layouts as lf_pool;
+ * every other entry is left untouched) and, when pool_q != 0, all of q_pool.
+ * Past KV frames do not change while a chunk denoises, so a caller that keeps
+ * k_pool / k_frame between calls of the same shape re-pools only the frames
+ * that changed (the current chunk) -- the pooled values are identical to a
+ * full lf_pool of the same k (per frame, the same arithmetic in the same
+ * order). The pages state that retrieval costs about 2 % of the run as history
+ * grows (paper.rainbus.top, limitations and conclusion); this is the persistent
+ * pooled-key cache that keeps the per-call pooling cost independent of the
+ * history length. Pointers, layouts and ownership as lf_pool; q may be NULL
+ * when pool_q == 0. Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE,
+ * LF_ERR_ARG (0 <= frame_begin <= frame_end <= n_frames violated), LF_ERR_CUDA.
+ */
+LF_API lf_status lf_pool_range(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                        int32_t frame_begin, int32_t frame_end, int32_t pool_q,
+                        float* q_pool, float* k_pool, float* k_frame, void* stream);
 
 /* Number of frames in each T_r: n_frames when chunk_index == 1, else
  * n_sink + min(topk_frames, n_mem) + n_recent + n_cur. Returns -1 on a bad shape. */

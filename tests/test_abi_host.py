@@ -142,6 +142,25 @@ def test_argument_validation():
     assert L.lib.lf_block_sparse_attn(S, p, p, p, p, p, 108, 0.0, mis, None) == 2
 
 
+def test_pool_range_validation():
+    sh = _shape()
+    p = ctypes.c_void_p(FAKE)
+    mis = ctypes.c_void_p(FAKE + 8)
+    S = ctypes.byref(sh)
+    nf = sh.n_frames
+    f = L.lib.lf_pool_range
+    assert f(S, p, p, -1, nf, 1, p, p, p, None) == 9          # frame_begin < 0
+    assert f(S, p, p, 3, 2, 1, p, p, p, None) == 9            # begin > end
+    assert f(S, p, p, 0, nf + 1, 1, p, p, p, None) == 9       # end past the last frame
+    assert f(S, None, p, 0, nf, 1, p, p, p, None) == 1        # q needed when pooling q
+    assert f(S, p, p, 0, nf, 1, None, p, p, None) == 1
+    assert f(S, None, p, 0, nf, 0, None, p, None, None) == 1   # k_frame always needed
+    assert f(S, None, mis, nf - 3, nf, 0, None, p, p, None) == 2  # q may be NULL without pool_q
+    assert f(None, p, p, 0, 1, 1, p, p, p, None) == 1
+    bad = _shape(head_dim=96)
+    assert f(ctypes.byref(bad), p, p, 0, 1, 1, p, p, p, None) == 3
+
+
 def test_status_strings():
     for code in range(12):
         assert L.lf_status_string(code)

@@ -114,3 +114,38 @@ def test_rollout_chunks():
         kb = shape.bpf if chunk == 1 else oracle.blocks_for_sparsity(s[chunk - 1], shape.Nkv, n_sel, shape.bpf)
         rows = parity.sample_rows(shape, per_block=2, blocks_per_head=3, seed=chunk)
         _full_check(shape, q, k, v, chunk, w.topk_frames, kb, rows=rows)
+
+
+def test_pool_range_reuses_past_frames():
+    """Pooled-key cache: after a full pooling of one chunk's keys, re-pooling only
+    the current-chunk frames of new keys gives exactly the full pooling of the new
+    keys (past frames untouched, same per-frame arithmetic), and both match the
+    oracle."""
+    import block_sparse_attention_lf_b200 as L
+    w = lf_synth.CONFIGS["layer480p"]
+    q, k, v = lf_synth.make_qkv(w)
+    shape = oracle.shape_of(w)
+    ls = L.shape_from_workload(w)
+    NF, C = ls.n_frames, ls.n_cur
+    k2 = k.clone()
+    F = ls.frame_tokens
+    g = torch.Generator().manual_seed(7)
+    k2[:, :, (NF - C) * F:, :] = torch.randn(k2[:, :, (NF - C) * F:, :].shape, generator=g).to(torch.bfloat16)
+    qd, kd, k2d = q.cuda(), k.cuda(), k2.cuda()
+    D = ls.head_dim
+    mk = lambda *s: torch.full(s, float("nan"), dtype=torch.float32, device="cuda")
+    qp, kp, kfr = mk(ls.batch, ls.heads, ls.Rq, D), mk(ls.batch, ls.heads, ls.Nkv, D), mk(ls.batch, ls.heads, NF, D)
+    L.lf_pool(ls, qd, kd, qp, kp, kfr)
+    L.lf_pool_range(ls, qd, k2d, NF - C, NF, qp, kp, kfr, pool_q=False)
+    qp2, kp2, kfr2 = mk(ls.batch, ls.heads, ls.Rq, D), mk(ls.batch, ls.heads, ls.Nkv, D), mk(ls.batch, ls.heads, NF, D)
+    L.lf_pool(ls, qd, k2d, qp2, kp2, kfr2)
+    torch.cuda.synchronize()
+    assert torch.equal(kp, kp2) and torch.equal(kfr, kfr2) and torch.equal(qp, qp2)
+    oq, ok, of = oracle.pool(shape, q, k2)
+    parity.check_pool({"q_pool": qp2.cpu().numpy(), "k_pool": kp2.cpu().numpy(), "k_frame": kfr2.cpu().numpy()},
+                      {"q_pool": oq, "k_pool": ok, "k_frame": of}, q, k2)
+    # an empty range leaves everything as it was
+    before = kp.clone()
+    L.lf_pool_range(ls, qd, kd, 3, 3, qp, kp, kfr, pool_q=False)
+    torch.cuda.synchronize()
+    assert torch.equal(before, kp)
