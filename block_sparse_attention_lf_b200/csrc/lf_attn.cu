@@ -38,11 +38,14 @@
 //     within m + 8 (p <= 256) is exponentiated against the current m; only when
 //     some row exceeds that bound does the warpgroup move m and rescale the
 //     matching O^T columns in TMEM.
-//   * Pipelines: three S buffers in TMEM (S runs up to three steps ahead), one
-//     P buffer (the warpgroups write it in step order), per-block V release.
-//     The MMA thread never blocks on one operand while another MMA is ready: it
-//     polls its barriers and issues whichever PV block (first) or S tile is
-//     ready.
+//   * Pipelines: three S buffers in TMEM, one P buffer (the warpgroups write it
+//     in step order), per-block V release. The MMA warp follows a static order --
+//     S of step s + 2, then PV of step s -- so the tensor pipe computes S(s+2)
+//     while the softmax turns S(s) into P(s). A single issuing warp has no other
+//     warp to hide its instruction latencies, so its per-step code path (waits,
+//     descriptors from precomputed bases, commits) is kept short: a polling
+//     scheduler that tested every barrier each round left the tensor pipe idle
+//     more than half of the time.
 //   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
@@ -316,98 +319,74 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer (whole warp,
-        // one elected lane issues; every branch below is warp-uniform)
+        // one elected lane issues). Static order: S of step s + 2, then PV of step s, so the
+        // tensor pipe computes S(s+2) while the softmax turns S(s) into P(s); the waits below
+        // are normally already satisfied, which keeps the issuing warp's code path short.
         {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, false);
-            const uint32_t sQ = smem_u32(smem + L::OFF_Q);
-            const uint32_t sK = smem_u32(smem + L::OFF_K);
-            const uint32_t sV = smem_u32(smem + L::OFF_V);
-            const uint32_t sP = smem_u32(smem + L::OFF_P);
+            // A descriptor's start field is the byte address >> 4, so an operand at a byte
+            // offset o from a base is the base descriptor + (o >> 4).
+            const uint64_t dQ = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
+            const uint64_t dK = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, L::K_SBO);
+            const uint64_t dV = sdesc_sw128(smem_u32(smem + L::OFF_V), L::V_LBO, L::V_SBO);
+            const uint64_t dP = sdesc_sw128(smem_u32(smem + L::OFF_P), 16, 1024);
             bool issued_any = false;
             bool ok = mbar_wait(&x.q_full, 0, abort_flag, a.err, 0x20);
-            int s_next = 0, s_half = 0;   // next S tile: step s_next, half s_half
-            int pv_next = 0, pv_blk = 0;  // next PV block: step pv_next, block pv_blk of 4
-            unsigned long long stall_t0 = 0;
-            uint32_t idle = 0;
-            while (ok && pv_next < n_steps) {
-                bool progressed = false;
-                // PV blocks of the oldest step whose P is written (frees V slots and, at the
-                // end of the step, the P buffer).
-                if (pv_next < s_next && mbar_test(&x.p_full, pv_next & 1)) {
-                    const int g = pv_next & 1;
-                    while (pv_blk < 4) {
-                        const int b = 4 * pv_next + pv_blk;
-                        if (b < cnt) {
-                            const int vs = b % VSLOTS;
-                            if (!mbar_test(&x.v_full[vs], (b / VSLOTS) & 1)) break;
-                            tc_fence_after();
+            // S of step st: A = Q (M = 64 queries, K-major), B = K tile (N = 128 keys, K-major),
+            // tile h of the step into TMEM lanes 16h.. of buffer st % SBUFS.
+            auto issue_s = [&](int st) -> bool {
+                const int bsel = st % SBUFS;
+                if (st >= SBUFS) {
+                    if (!mbar_wait(&x.s_free[bsel], ((st / SBUFS) - 1) & 1, abort_flag, a.err, 0x21)) return false;
+                    tc_fence_after();  // the softmax's TMEM reads of this buffer come first
+                }
+                for (int h = 0; h < 2; ++h) {
+                    const int t = 2 * st + h;
+                    if (t >= n_tiles) break;
+                    const int ks = t % KSLOTS;
+                    if (!mbar_wait(&x.k_full[ks], (t / KSLOTS) & 1, abort_flag, a.err, 0x22)) return false;
+                    const uint32_t d_addr = tmem + 128u * static_cast<uint32_t>(bsel) + (h ? (16u << 16) : 0u);
+                    const uint64_t kb = dK + ((static_cast<uint32_t>(ks) * L::K_SLOT) >> 4);
 #pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4) {
-                                // A = V_block^T (M = head_dim, MN-major), B = P^T (N = 64 queries, K-major)
-                                const uint64_t ad = sdesc_sw128(sV + vs * L::V_SLOT + k4 * L::V_K16, L::V_LBO, L::V_SBO);
-                                const uint64_t bd = sdesc_sw128(sP + pv_blk * L::P_PANEL + k4 * 32, 16, 1024);
-                                umma_bf16_elect(tmem + TM_O + 64u * g, ad, bd, IDESC_O,
-                                          (pv_next >= 2 || pv_blk > 0 || k4 > 0) ? 1u : 0u);
-                            }
-                            umma_commit_elect(&x.v_empty[vs]);
-                            issued_any = true;
-                        }
-                        ++pv_blk;
-                        progressed = true;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oq = ((kk >> 2) * L::PANEL_Q + (kk & 3) * 32) >> 4;
+                        const uint32_t ok_ = ((kk >> 2) * L::K_PANEL + (kk & 3) * 32) >> 4;
+                        umma_bf16_elect(d_addr, dQ + oq, kb + ok_, IDESC_S, kk > 0 ? 1u : 0u);
                     }
-                    if (pv_blk == 4) {
-                        umma_commit_elect(&x.p_empty[pv_next & 1]);
-                        ++pv_next;
-                        pv_blk = 0;
-                    }
+                    umma_commit_elect(&x.k_empty[ks]);
+                    issued_any = true;
                 }
-                // S tiles: step s_next needs its TMEM buffer free and its K tile landed.
-                // S runs at most two steps ahead of the oldest PV not yet issued, so that
-                // a PV whose P is written does not queue behind more S work.
-                if (s_next < n_steps && s_next <= pv_next + 2) {
-                    const int bsel = s_next % SBUFS;
-                    const int t = 2 * s_next + s_half;
-                    const bool buf_free =
-                        s_half == 1 || s_next < SBUFS || mbar_test(&x.s_free[bsel], ((s_next / SBUFS) - 1) & 1);
-                    // (t < n_tiles always: a step with an empty second half ends after its first)
-                    if (buf_free && mbar_test(&x.k_full[t % KSLOTS], (t / KSLOTS) & 1)) {
-                        tc_fence_after();
-                        const uint32_t ks = static_cast<uint32_t>(t % KSLOTS);
-                        const uint32_t d_addr = tmem + 128u * bsel + (s_half ? (16u << 16) : 0u);
+                umma_commit_elect(&x.s_full[bsel]);
+                return true;
+            };
+            // PV of step st: A = V block^T (M = head_dim, MN-major), B = P^T (N = 64 queries,
+            // K-major), into O^T of warpgroup st % 2; V slots are released block by block.
+            auto issue_pv = [&](int st) -> bool {
+                if (!mbar_wait(&x.p_full, st & 1, abort_flag, a.err, 0x23)) return false;
+                tc_fence_after();  // an O^T rescale by the softmax comes first
+                const uint32_t d_addr = tmem + TM_O + 64u * static_cast<uint32_t>(st & 1);
+                for (int q = 0; q < 4; ++q) {
+                    const int b = 4 * st + q;
+                    if (b >= cnt) break;
+                    const int vs = b % VSLOTS;
+                    if (!mbar_wait(&x.v_full[vs], (b / VSLOTS) & 1, abort_flag, a.err, 0x24)) return false;
+                    const uint64_t vb = dV + ((static_cast<uint32_t>(vs) * L::V_SLOT) >> 4);
+                    const uint64_t pb = dP + ((static_cast<uint32_t>(q) * L::P_PANEL) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t panel = static_cast<uint32_t>(kk >> 2);
-                            // A = Q (M = 64 queries, K-major), B = K tile (N = 128 keys, K-major)
-                            const uint64_t ad = sdesc_sw128(sQ + panel * L::PANEL_Q + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd =
-                                sdesc_sw128(sK + ks * L::K_SLOT + panel * L::K_PANEL + (kk & 3) * 32, 16, L::K_SBO);
-                            umma_bf16_elect(d_addr, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit_elect(&x.k_empty[ks]);
-                        issued_any = true;
-                        if (s_half == 1 || t + 1 >= n_tiles) {
-                            umma_commit_elect(&x.s_full[bsel]);
-                            ++s_next;
-                            s_half = 0;
-                        } else {
-                            s_half = 1;
-                        }
-                        progressed = true;
-                    }
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        umma_bf16_elect(d_addr, vb + ((k4 * L::V_K16) >> 4), pb + ((k4 * 32) >> 4), IDESC_O,
+                                        (st >= 2 || q > 0 || k4 > 0) ? 1u : 0u);
+                    umma_commit_elect(&x.v_empty[vs]);
+                    issued_any = true;
                 }
-                if (progressed) {
-                    idle = 0;
-                } else if (++idle == 1) {
-                    stall_t0 = globaltimer();
-                } else if ((idle & 63u) == 0u) {
-                    if (*abort_flag) break;
-                    if (globaltimer() - stall_t0 > LF_WAIT_LIMIT_NS) {
-                        *abort_flag = 1;
-                        record_error(a.err, DEVERR_TIMEOUT | 0x22);
-                        break;
-                    }
-                }
+                umma_commit_elect(&x.p_empty[st & 1]);
+                return true;
+            };
+            for (int st = 0; ok && st < min(2, n_steps); ++st) ok = issue_s(st);
+            for (int st = 0; ok && st < n_steps; ++st) {
+                if (st + 2 < n_steps) ok = issue_s(st + 2);
+                if (ok) ok = issue_pv(st);
             }
             if (*abort_flag && issued_any) {
                 umma_commit_elect(&x.drain);
