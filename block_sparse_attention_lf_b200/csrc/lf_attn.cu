@@ -26,7 +26,7 @@
 //     MN-major (LBO = 1 KB between head-dim panels, SBO = 2 KB between 8-row
 //     groups). Frames whose token count is not a multiple of 8, and head_dim
 //     64, use 2-D boxes per 64-wide panel into a plain [panel][row] layout.
-//     K arrives per tile (ring of 3 tiles), V per block (ring of 4 blocks).
+//     K arrives per tile (ring of 2 tiles), V per block (ring of 4 blocks).
 //   * Warp roles (384 threads): warp 0 issues the Q and K loads, warp 1 the V
 //     loads, warp 2 allocates TMEM and issues tcgen05.mma from one thread,
 //     warp 3 idles, warps 4-11 are two softmax warpgroups. Warpgroup g takes
@@ -38,8 +38,9 @@
 //     within m + 8 (p <= 256) is exponentiated against the current m; only when
 //     some row exceeds that bound does the warpgroup move m and rescale the
 //     matching O^T columns in TMEM.
-//   * Pipelines: three S buffers in TMEM, one P buffer (the warpgroups write it
-//     in step order), per-block V release. The MMA warp follows a static order --
+//   * Pipelines: three S buffers in TMEM, a P buffer per warpgroup (a warpgroup
+//     rewrites its P once the PV of its previous step is done), per-block V
+//     release. The MMA warp follows a static order --
 //     S of step s + 2, then PV of step s -- so the tensor pipe computes S(s+2)
 //     while the softmax turns S(s) into P(s). A single issuing warp has no other
 //     warp to hide its instruction latencies, so its per-step code path (waits,
@@ -62,7 +63,7 @@ namespace {
 
 constexpr int ATTN_THREADS = 384;
 constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_SOFT0 = 4;
-constexpr int KSLOTS = 3;   // K ring: tiles of two blocks
+constexpr int KSLOTS = 2;   // K ring: tiles of two blocks
 constexpr int VSLOTS = 4;   // V ring: single blocks
 constexpr int SBUFS = 3;    // S buffers in TMEM (one per step in flight)
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
@@ -86,7 +87,7 @@ struct AttnLayout {
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + KSLOTS * K_SLOT;
     static constexpr uint32_t OFF_P = OFF_V + VSLOTS * V_SLOT;
-    static constexpr uint32_t OFF_AUX = OFF_P + P_BYTES;
+    static constexpr uint32_t OFF_AUX = OFF_P + 2 * P_BYTES;
     // K tile (B operand of the S MMA, K-major): 8-row group stride and panel offset
     static constexpr uint32_t K_SBO = IL ? 2048u : 1024u;
     static constexpr uint32_t K_PANEL = IL ? 1024u : 128u * 128u;
@@ -103,7 +104,7 @@ struct AttnAux {
     uint64_t k_full[KSLOTS], k_empty[KSLOTS];
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
     uint64_t s_full[SBUFS], s_free[SBUFS];
-    uint64_t p_full, p_empty[2];
+    uint64_t p_full[2], p_empty[2];  // per warpgroup: its P written / its last PV done
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -224,7 +225,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             mbar_init(&x.s_full[s], 1);
             mbar_init(&x.s_free[s], 4);  // one arrival per warp of the owning warpgroup
         }
-        mbar_init(&x.p_full, 4);
+        mbar_init(&x.p_full[0], 4);
+        mbar_init(&x.p_full[1], 4);
         mbar_init(&x.p_empty[0], 1);
         mbar_init(&x.p_empty[1], 1);
         mbar_init(&x.drain, 1);
@@ -363,7 +365,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             // PV of step st: A = V block^T (M = head_dim, MN-major), B = P^T (N = 64 queries,
             // K-major), into O^T of warpgroup st % 2; V slots are released block by block.
             auto issue_pv = [&](int st) -> bool {
-                if (!mbar_wait(&x.p_full, st & 1, abort_flag, a.err, 0x23)) return false;
+                if (!mbar_wait(&x.p_full[st & 1], (st >> 1) & 1, abort_flag, a.err, 0x23)) return false;
                 tc_fence_after();  // an O^T rescale by the softmax comes first
                 const uint32_t d_addr = tmem + TM_O + 64u * static_cast<uint32_t>(st & 1);
                 for (int q = 0; q < 4; ++q) {
@@ -372,7 +374,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const int vs = b % VSLOTS;
                     if (!mbar_wait(&x.v_full[vs], (b / VSLOTS) & 1, abort_flag, a.err, 0x24)) return false;
                     const uint64_t vb = dV + ((static_cast<uint32_t>(vs) * L::V_SLOT) >> 4);
-                    const uint64_t pb = dP + ((static_cast<uint32_t>(q) * L::P_PANEL) >> 4);
+                    const uint64_t pb = dP + ((static_cast<uint32_t>(st & 1) * L::P_BYTES + static_cast<uint32_t>(q) * L::P_PANEL) >> 4);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
                         umma_bf16_elect(d_addr, vb + ((k4 * L::V_K16) >> 4), pb + ((k4 * 32) >> 4), IDESC_O,
@@ -404,7 +406,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const uint32_t o_col = TM_O + 64u * static_cast<uint32_t>(g);
         const float sl2 = a.scale_log2;
         // this thread's P row: panels 2*hh and 2*hh+1 (keys 128*hh ... 128*hh+127 of the step)
-        uint8_t* prow = smem + L::OFF_P + (2 * hh) * L::P_PANEL + qr * 128;
+        uint8_t* prow = smem + L::OFF_P + g * L::P_BYTES + (2 * hh) * L::P_PANEL + qr * 128;
         float m_run = -INFINITY;  // stabiliser of this row (identical in lanes l and l^16)
         float l_run = 0.f;        // this thread's share of the row's softmax denominator
 
@@ -453,8 +455,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float alpha = need ? fast_exp2(m_run - m_new) : 1.f;  // 0 when m_run = -inf
             l_run *= alpha;
             m_run = m_new;
-            // 2. Probabilities (registers), then wait until PV of the previous step
-            // has read the P buffer (it also ends this warpgroup's last PV).
+            // 2. Probabilities (registers), then wait until the PV of this warpgroup's
+            // previous step has read its P buffer and finished accumulating into its O^T.
             const float mu = (m_run == -INFINITY) ? 0.f : m_run;
             uint32_t pk[64];
             float la = 0.f, lb = 0.f;
@@ -468,7 +470,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 pk[c >> 1] = pack_bf16x2(p0, p1);
             }
             l_run += la + lb;
-            if (s > 0) mbar_wait(&x.p_empty[(s - 1) & 1], ((s - 1) >> 1) & 1, abort_flag, a.err, 0x31);
+            if (j > 0) mbar_wait(&x.p_empty[g], (j - 1) & 1, abort_flag, a.err, 0x31);
             // 3. P row -> shared memory (two 64-key panels, 128-byte swizzle).
 #pragma unroll
             for (int pp = 0; pp < 2; ++pp) {
@@ -508,7 +510,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&x.p_full);
+            if (lane == 0) mbar_arrive(&x.p_full[g]);
         }
 
         // ------------------------------------------------------------ epilogue
@@ -518,8 +520,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             x.m_s[g][qr] = m_run;
         }
         // the last PV of the call ends every PV of both warpgroups
-        if (n_steps > 0)
-            mbar_wait(&x.p_empty[(n_steps - 1) & 1], ((n_steps - 1) >> 1) & 1, abort_flag, a.err, 0x34);
+        if (j > 0) mbar_wait(&x.p_empty[g], (j - 1) & 1, abort_flag, a.err, 0x34);
         tc_fence_before();
         named_bar_sync(3, 256);  // both warpgroups: sums, maxima and last PVs are final
         tc_fence_after();
