@@ -28,8 +28,8 @@
 //     64, use 2-D boxes per 64-wide panel into a plain [panel][row] layout.
 //     K arrives per tile (ring of 2 tiles), V per block (ring of 4 blocks).
 //   * Warp roles (384 threads): warp 0 issues the Q and K loads, warp 1 the V
-//     loads, warp 2 allocates TMEM and issues tcgen05.mma from one thread,
-//     warp 3 idles, warps 4-11 are two softmax warpgroups. Warpgroup g takes
+//     loads, warp 2 allocates TMEM and issues the score MMAs, warp 3 issues the
+//     PV MMAs, warps 4-11 are two softmax warpgroups. Warpgroup g takes
 //     the steps s with s % 2 == g, with its own running maxima and its own O^T
 //     accumulator in TMEM; the two partial softmaxes are merged once in the
 //     epilogue (O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M))).
@@ -40,13 +40,15 @@
 //     matching O^T columns in TMEM.
 //   * Pipelines: three S buffers in TMEM, a P buffer per warpgroup (a warpgroup
 //     rewrites its P once the PV of its previous step is done), per-block V
-//     release. The MMA warp follows a static order --
-//     S of step s + 2, then PV of step s -- so the tensor pipe computes S(s+2)
-//     while the softmax turns S(s) into P(s). A single issuing warp has no other
-//     warp to hide its instruction latencies, so its per-step code path (waits,
-//     descriptors from precomputed bases, commits) is kept short: a polling
-//     scheduler that tested every barrier each round left the tensor pipe idle
-//     more than half of the time.
+//     release. Two MMA warps, each in step order with blocking waits: one issues
+//     the score MMAs (up to three steps ahead, bounded by the S buffers), the
+//     other the PV MMAs; their commits track only their own MMAs and no
+//     ordering between the two streams is needed (the S and O^T regions are
+//     disjoint, a warpgroup only waits for its own PVs). A lone issuing warp has
+//     no other warp to hide its instruction latencies, so each warp's per-step
+//     code path (waits, descriptors from precomputed bases, commits) is kept
+//     short: a single polling scheduler that tested every barrier each round
+//     left the tensor pipe idle more than half of the time.
 //   * Every mbarrier wait is bounded (1 s); on expiry the CTA sets an abort
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
@@ -62,7 +64,7 @@ namespace lf {
 namespace {
 
 constexpr int ATTN_THREADS = 384;
-constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_SOFT0 = 4;
+constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_PV = 3, W_SOFT0 = 4;
 constexpr int KSLOTS = 2;   // K ring: tiles of two blocks
 constexpr int VSLOTS = 4;   // V ring: single blocks
 constexpr int SBUFS = 3;    // S buffers in TMEM (one per step in flight)
@@ -105,7 +107,7 @@ struct AttnAux {
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
     uint64_t s_full[SBUFS], s_free[SBUFS];
     uint64_t p_full[2], p_empty[2];  // per warpgroup: its P written / its last PV done
-    uint64_t drain;
+    uint64_t drain, drain_pv;
     uint32_t tmem_base;
     int abort;
     alignas(16) float alpha[2][64];  // per-warpgroup rescale factors of the query columns
@@ -230,6 +232,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(&x.p_empty[0], 1);
         mbar_init(&x.p_empty[1], 1);
         mbar_init(&x.drain, 1);
+        mbar_init(&x.drain_pv, 1);
         x.abort = 0;
         fence_mbar_init();
     }
@@ -319,11 +322,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int b = max(0, armed - VSLOTS); b < armed; ++b)
                     mbar_drain(&x.v_full[b % VSLOTS], (b / VSLOTS) & 1, 10000000ull);
         }
-    } else if (warp == W_MMA) {
-        // ------------------------------------------------------------ MMA issuer (whole warp,
-        // one elected lane issues). Static order: S of step s + 2, then PV of step s, so the
-        // tensor pipe computes S(s+2) while the softmax turns S(s) into P(s); the waits below
-        // are normally already satisfied, which keeps the issuing warp's code path short.
+    } else if (warp == W_MMA || warp == W_PV) {
+        // ------------------------------------------------------------ MMA issuers (whole warps,
+        // one elected lane issues): warp W_MMA issues the score MMAs of every step in order,
+        // warp W_PV the PV MMAs; the waits below are normally already satisfied, which keeps
+        // each issuing warp's code path short.
         {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, false);
@@ -385,14 +388,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 umma_commit_elect(&x.p_empty[st & 1]);
                 return true;
             };
-            for (int st = 0; ok && st < min(2, n_steps); ++st) ok = issue_s(st);
-            for (int st = 0; ok && st < n_steps; ++st) {
-                if (st + 2 < n_steps) ok = issue_s(st + 2);
-                if (ok) ok = issue_pv(st);
+            if (warp == W_MMA) {
+                for (int st = 0; ok && st < n_steps; ++st) ok = issue_s(st);
+            } else {
+                for (int st = 0; ok && st < n_steps; ++st) ok = issue_pv(st);
             }
             if (*abort_flag && issued_any) {
-                umma_commit_elect(&x.drain);
-                mbar_drain(&x.drain, 0, 10000000ull);
+                uint64_t* dr = warp == W_MMA ? &x.drain : &x.drain_pv;
+                umma_commit_elect(dr);
+                mbar_drain(dr, 0, 10000000ull);
             }
         }
     } else if (warp >= W_SOFT0) {
