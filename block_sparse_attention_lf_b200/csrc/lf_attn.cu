@@ -113,6 +113,7 @@ struct AttnAux {
     alignas(16) float alpha[2][64];  // per-warpgroup rescale factors of the query columns
     float lsum[2][64];               // softmax denominators of each warpgroup's rows
     alignas(16) float m_s[2][64];    // final running max (log2 units) per warpgroup and query row
+    float wgt[2][64];                // epilogue weights of the two accumulators per query row
     int lst[LIST_SMEM];              // the CTA's block list (entries past LIST_SMEM stay in global memory)
 };
 
@@ -534,20 +535,29 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncwarp();
         tmem_ld32(lane_base + TM_O + 32u * g, o0);
         tmem_ld32(lane_base + TM_O + 64u + 32u * g, o1);
-        tmem_ld_wait();
         __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K);
         const int t = sp * 32 + lane;
+        // O = O_0 w_0 + O_1 w_1 with w_i = 2^(m_i - M) / l: one division and two
+        // exponentials per query row, by the first warp of the warpgroup
+        if (t < 32) {
+            const int cc = 32 * g + t;
+            const float m0 = x.m_s[0][cc], m1 = x.m_s[1][cc];
+            const float mx = fmaxf(m0, m1);
+            const float f0 = (n0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - mx) : 0.f;
+            const float f1 = (n1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - mx) : 0.f;
+            const float den = x.lsum[0][cc] * f0 + x.lsum[1][cc] * f1;
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            x.wgt[0][cc] = f0 * inv;
+            x.wgt[1][cc] = f1 * inv;
+        }
+        tmem_ld_wait();
+        named_bar_sync(bar_id, 128);  // this warpgroup's weights are visible
         if (t < D) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 const int cc = 32 * g + c;
-                const float m0 = x.m_s[0][cc], m1 = x.m_s[1][cc];
-                const float mx = fmaxf(m0, m1);
-                const float f0 = (n0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - mx) : 0.f;
-                const float f1 = (n1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - mx) : 0.f;
-                const float den = x.lsum[0][cc] * f0 + x.lsum[1][cc] * f1;
-                const float num = (f0 != 0.f ? o0[c] * f0 : 0.f) + (f1 != 0.f ? o1[c] * f1 : 0.f);
-                ostage[cc * D + t] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+                const float w0 = x.wgt[0][cc], w1 = x.wgt[1][cc];
+                ostage[cc * D + t] = __float2bfloat16_rn((w0 != 0.f ? o0[c] * w0 : 0.f) + (w1 != 0.f ? o1[c] * w1 : 0.f));
             }
         }
         named_bar_sync(3, 256);
