@@ -519,7 +519,7 @@ def run_ours(a):
                      "peak_source": f"{peaks['source']} bf16 dense burst (MEASURED_PEAKS.json)"},
         "e2e": {"value": ws * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e},
-        "gpu_launches": 4 * a.steps,
+        "gpu_launches": call.launches_per_call * a.steps,
         "clocks": clk.summary(),
         "wall_s_timed_region": wall,
     }

@@ -25,16 +25,17 @@ LIB_PATH = os.path.join(_HERE, "liblf_hsa.so")
 
 __all__ = [
     "LfShape", "LfError", "lib", "lf_pool", "lf_pool_range", "lf_select_frames", "lf_select_blocks",
-    "lf_block_sparse_attn", "lf_cag_budget", "lf_blocks_for_sparsity", "lf_frames_selected",
-    "lf_list_capacity", "lf_get_device_error", "lf_status_string", "lf_version", "HSACall",
+    "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
+    "lf_blocks_for_sparsity", "lf_frames_selected", "lf_list_capacity", "lf_get_device_error",
+    "lf_status_string", "lf_version", "HSACall",
     "ABI_FUNCTIONS",
 ]
 
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
     "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
-    "lf_block_sparse_attn", "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error",
-    "lf_status_string", "lf_version",
+    "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
+    "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
 )
 
 LF_OK = 0
@@ -104,6 +105,9 @@ def _load() -> ctypes.CDLL:
         "lf_list_capacity": ([S, I32, I32, I32], I32),
         "lf_select_blocks": ([S, I32, I32, I32, P, P, P, P, P, I32, P], I32),
         "lf_block_sparse_attn": ([S, P, P, P, P, P, I32, F32, P, P], I32),
+        "lf_block_sparse_attn_ws": ([S, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
+        "lf_attn_split_plan": ([S, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
+                                ctypes.POINTER(ctypes.c_int64)], I32),
         "lf_cag_budget": ([I32, P, P, F64, F64, I32, P, P], I32),
         "lf_blocks_for_sparsity": ([F64, I32, I32, I32], I32),
         "lf_get_device_error": ([ctypes.POINTER(I32)], I32),
@@ -227,6 +231,31 @@ def lf_block_sparse_attn(shape: LfShape, q, k, v, block_list, block_count, list_
            "lf_block_sparse_attn")
 
 
+def lf_block_sparse_attn_ws(shape: LfShape, q, k, v, block_list, block_count, list_cap: int,
+                            softmax_scale: float, out, workspace=None, tail_pieces: int = 0,
+                            stream=None) -> None:
+    """``workspace``: a uint8 device tensor (or None: no split)."""
+    import torch
+    bf = _bf16()
+    ws = _dev_ptr(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(_lib.lf_block_sparse_attn_ws(ctypes.byref(shape), _dev_ptr(q, bf, "q"), _dev_ptr(k, bf, "k"),
+                                        _dev_ptr(v, bf, "v"),
+                                        _dev_ptr(block_list, torch.int32, "block_list"),
+                                        _dev_ptr(block_count, torch.int32, "block_count"), list_cap,
+                                        float(softmax_scale), _dev_ptr(out, bf, "out"), int(tail_pieces),
+                                        ws, ws_bytes, _stream(stream)),
+           "lf_block_sparse_attn_ws")
+
+
+def lf_attn_split_plan(shape: LfShape, list_cap: int, sm: int = 0) -> Tuple[int, int, int]:
+    """(tail query blocks, pieces per list, workspace bytes) of the automatic split."""
+    t, p, b = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int64(0)
+    _check(_lib.lf_attn_split_plan(ctypes.byref(shape), list_cap, sm, ctypes.byref(t), ctypes.byref(p),
+                                   ctypes.byref(b)), "lf_attn_split_plan")
+    return t.value, p.value, b.value
+
+
 def lf_cag_budget(T: Sequence[float], flops_w: Optional[Sequence[float]], s_base: float,
                   s_target: float, target_over_all: bool = True) -> Tuple[int, list, float]:
     """Host-only Chunk-Aware Growth solver: returns (status, s[n], beta)."""
@@ -265,11 +294,14 @@ class HSACall:
     """One HSA call's device buffers plus the four device steps, in order.
 
     ``shape``: an ``LfShape``; ``chunk_index`` is 1-based (chunk 1 is dense);
-    ``topk_frames`` / ``topk_blocks`` as in the C ABI.
+    ``topk_frames`` / ``topk_blocks`` as in the C ABI. ``tail_pieces`` selects
+    the attention's split of the last, partial wave (0: automatic plan for the
+    current device, 1: none, k >= 2: k pieces); the workspace it needs is
+    allocated here.
     """
 
     def __init__(self, shape: LfShape, chunk_index: int, topk_frames: int, topk_blocks: int,
-                 device="cuda", softmax_scale: float = 0.0):
+                 device="cuda", softmax_scale: float = 0.0, tail_pieces: int = 0):
         import torch
         self.shape, self.chunk_index = shape, chunk_index
         self.topk_frames, self.topk_blocks = topk_frames, topk_blocks
@@ -292,6 +324,23 @@ class HSACall:
             out=torch.empty(s.batch, s.heads, s.Lq, D, dtype=torch.bfloat16, device=device),
             list_cap=cap,
         )
+        self.tail_pieces = tail_pieces
+        if tail_pieces == 0:
+            tail, pieces, _ = lf_attn_split_plan(s, cap)
+        elif tail_pieces >= 2:
+            # the same tail as the automatic plan, with the piece count given
+            sm = torch.cuda.get_device_properties(torch.device(device)).multi_processor_count
+            tail = (s.batch * s.heads * s.Rq) % sm
+            pieces = min(tail_pieces, cap)
+            if pieces < 2:
+                tail, pieces = 0, 0
+        else:
+            tail, pieces = 0, 0
+        ws_bytes = tail * pieces * 64 * (D + 2) * 4
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes else None
+        self.split = (tail, pieces) if ws_bytes else (0, 0)
+        # kernels enqueued per call: pool, two selections, attention (+ the merge of a split)
+        self.launches_per_call = 4 + (1 if ws_bytes else 0)
 
     def pool(self, q, k, stream=None):
         b = self.buf
@@ -306,8 +355,8 @@ class HSACall:
 
     def attend(self, q, k, v, stream=None):
         b = self.buf
-        lf_block_sparse_attn(self.shape, q, k, v, b.block_list, b.block_count, b.list_cap,
-                             self.softmax_scale, b.out, stream)
+        lf_block_sparse_attn_ws(self.shape, q, k, v, b.block_list, b.block_count, b.list_cap,
+                                self.softmax_scale, b.out, self.workspace, self.tail_pieces, stream)
 
     def __call__(self, q, k, v, stream=None):
         self.pool(q, k, stream)

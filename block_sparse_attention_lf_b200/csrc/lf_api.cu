@@ -5,6 +5,7 @@
 #include "lf_device.cuh"
 #include "lf_internal.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -94,6 +95,44 @@ int blocks_per_frame(const Derived& d, int chunk_index, int topk_blocks)
 }
 
 lf_status launch_status(cudaError_t e) { return e == cudaSuccess ? LF_OK : LF_ERR_CUDA; }
+
+// Bytes of one partial-result slot of the attention split: 64 rows of head_dim
+// fp32 values plus a (max, denominator) pair per row.
+long long split_slot_bytes(int D) { return 64ll * (D + 2) * 4; }
+
+// Split of the last, partial wave of the one-CTA-per-query-block attention.
+// With n_rows query blocks on sm SMs, the last r = n_rows mod sm query blocks
+// (all of them when n_rows < sm) would run as a wave of r CTAs on r SMs; their
+// lists are cut into k pieces instead. Automatic k (force == 0): sm / r, at most
+// list_cap / 8 (a piece of a full list keeps two steps), and no split when sm / r
+// is below 8: with the last wave filling more than an eighth of the SMs the
+// pieces' own set-up and the merge cost about what the split saves (measured:
+// 12 of 148 SMs 344 -> 333 us, 24 of 148 SMs 648 -> 646 and 377 -> 382 us).
+// force == 1: no split; force >= 2: k = force. k is capped at list_cap and at
+// the slots the workspace holds (slots_cap < 0: unlimited); k < 2: no split.
+void split_plan(long long n_rows, int sm, int list_cap, int force, long long slots_cap, int* tail, int* pieces)
+{
+    *tail = 0;
+    *pieces = 0;
+    if (n_rows <= 0 || sm <= 0 || force == 1) return;
+    const long long r = n_rows % sm;
+    if (r == 0) return;
+    long long k = force >= 2 ? force : std::min<long long>(sm / r, list_cap / 8);
+    if (force == 0 && sm / r < 8) return;
+    k = std::min<long long>(k, list_cap);
+    if (slots_cap >= 0) k = std::min(k, slots_cap / r);
+    if (k < 2) return;
+    *tail = static_cast<int>(r);
+    *pieces = static_cast<int>(k);
+}
+
+lf_status sm_count(int* out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    if (cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    return LF_OK;
+}
 
 // ---- TMA descriptors ------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -243,18 +282,46 @@ lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index, int32
     return launch_status(lf::launch_select_blocks(a, static_cast<cudaStream_t>(stream)));
 }
 
+lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap, int32_t sm, int32_t* tail_rows,
+                             int32_t* pieces, int64_t* workspace_bytes)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (list_cap < 0) return LF_ERR_CAP;
+    if (!tail_rows || !pieces || !workspace_bytes) return LF_ERR_NULL;
+    if (sm <= 0 && (st = sm_count(&sm)) != LF_OK) return st;
+    int t = 0, kp = 0;
+    split_plan(static_cast<long long>(d.B) * d.H * d.Rq, sm, list_cap, 0, -1, &t, &kp);
+    *tail_rows = t;
+    *pieces = kp;
+    *workspace_bytes = static_cast<int64_t>(t) * kp * split_slot_bytes(d.D);
+    return LF_OK;
+}
+
 lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                const int32_t* block_list, const int32_t* block_count, int32_t list_cap,
                                float softmax_scale, uint16_t* out, void* stream)
+{
+    return lf_block_sparse_attn_ws(shape, q, k, v, block_list, block_count, list_cap, softmax_scale, out, 1, nullptr,
+                                   0, stream);
+}
+
+lf_status lf_block_sparse_attn_ws(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                  const int32_t* block_list, const int32_t* block_count, int32_t list_cap,
+                                  float softmax_scale, uint16_t* out, int32_t tail_pieces, void* workspace,
+                                  int64_t workspace_bytes, void* stream)
 {
     Derived d;
     lf_status st = check_shape(shape, &d);
     if (st != LF_OK) return st;
     if (list_cap < 0) return LF_ERR_CAP;
     if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return LF_ERR_ARG;
+    if (tail_pieces < 0 || workspace_bytes < 0) return LF_ERR_ARG;
     if (!q || !k || !v || !block_list || !block_count || !out) return LF_ERR_NULL;
+    if (workspace_bytes > 0 && !workspace) return LF_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_list) || !aligned16(block_count) ||
-        !aligned16(out))
+        !aligned16(out) || (workspace_bytes > 0 && !aligned16(workspace)))
         return LF_ERR_ALIGN;
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
@@ -277,10 +344,19 @@ lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t* q, con
         (!encode_rows(&m.k, k, kv_rows, d.D, 64) || !encode_rows(&m.k_rem, k, kv_rows, d.D, d.rem) ||
          !encode_rows(&m.v, v, kv_rows, d.D, 64) || !encode_rows(&m.v_rem, v, kv_rows, d.D, d.rem)))
         return LF_ERR_CUDA;
+    const long long n_rows = BH * d.Rq;
+    int tail = 0, pieces = 0;
+    if (workspace_bytes > 0 && tail_pieces != 1) {
+        int sm = 0;
+        if ((st = sm_count(&sm)) != LF_OK) return st;
+        split_plan(n_rows, sm, list_cap, tail_pieces, workspace_bytes / split_slot_bytes(d.D), &tail, &pieces);
+    }
+    float* part_o = static_cast<float*>(workspace);
+    float* part_ml = pieces ? part_o + static_cast<long long>(tail) * pieces * 64 * d.D : nullptr;
     lf::AttnArgs a{block_list, block_count, out, list_cap, d.Rq, d.bpf, d.F, d.Lq, d.Nkv, d.rem, d.kv_stride,
-                   scale * 1.4426950408889634f, err};
+                   scale * 1.4426950408889634f, err, static_cast<int>(n_rows - tail), pieces, part_o, part_ml};
     return launch_status(
-        lf::launch_attn(m, a, d.D, interleaved, static_cast<int>(BH * d.Rq), static_cast<cudaStream_t>(stream)));
+        lf::launch_attn(m, a, d.D, interleaved, static_cast<int>(n_rows), static_cast<cudaStream_t>(stream)));
 }
 
 lf_status lf_cag_budget(int32_t n_chunks, const double* T, const double* flops_w, double s_base, double s_target,

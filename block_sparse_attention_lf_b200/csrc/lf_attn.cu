@@ -204,7 +204,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     AttnAux& x = *reinterpret_cast<AttnAux*>(smem + L::OFF_AUX);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row = blockIdx.x;
+    // the merge kernel of a split call may be scheduled once every CTA has started
+    // (it waits for this grid's completion before reading anything)
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    int row = blockIdx.x;
+    int slot = -1;  // partial-result slot of a CTA that computes one piece of a list
+    if (a.pieces > 0 && row >= a.n_whole) {
+        slot = row - a.n_whole;
+        row = a.n_whole + slot / a.pieces;
+    }
     const int bh = row / a.Rq;
     const int r = row - bh * a.Rq;
     int cnt = __ldg(a.block_count + row);
@@ -213,6 +221,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         cnt = cnt < 0 ? 0 : a.list_cap;
     }
     const int* lst = a.block_list + static_cast<long long>(row) * a.list_cap;
+    if (slot >= 0) {
+        // entries [piece * cnt / pieces, (piece + 1) * cnt / pieces) of the list
+        const int piece = slot % a.pieces;
+        const int lo = static_cast<int>(static_cast<long long>(piece) * cnt / a.pieces);
+        const int hi = static_cast<int>(static_cast<long long>(piece + 1) * cnt / a.pieces);
+        lst += lo;
+        cnt = hi - lo;
+    }
     const int n_tiles = (cnt + 1) >> 1;
     const int n_steps = (n_tiles + 1) >> 1;
     const int fq = r / a.bpf;
@@ -549,24 +565,43 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float inv = den > 0.f ? 1.f / den : 0.f;
             x.wgt[0][cc] = f0 * inv;
             x.wgt[1][cc] = f1 * inv;
+            if (slot >= 0) {
+                float* ml = a.part_ml + (static_cast<long long>(slot) * 64 + cc) * 2;
+                ml[0] = den > 0.f ? mx : -INFINITY;
+                ml[1] = den > 0.f ? den : 0.f;
+            }
         }
         tmem_ld_wait();
         named_bar_sync(bar_id, 128);  // this warpgroup's weights are visible
-        if (t < D) {
+        if (slot >= 0) {
+            // one piece of a list: normalised fp32 rows for the merge kernel (a warp
+            // stores 32 consecutive floats of one row at a time)
+            if (t < D) {
+                float* po = a.part_o + static_cast<long long>(slot) * 64 * D + t;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int cc = 32 * g + c;
-                const float w0 = x.wgt[0][cc], w1 = x.wgt[1][cc];
-                ostage[cc * D + t] = __float2bfloat16_rn((w0 != 0.f ? o0[c] * w0 : 0.f) + (w1 != 0.f ? o1[c] * w1 : 0.f));
+                for (int c = 0; c < 32; ++c) {
+                    const int cc = 32 * g + c;
+                    const float w0 = x.wgt[0][cc], w1 = x.wgt[1][cc];
+                    po[static_cast<long long>(cc) * D] = (w0 != 0.f ? o0[c] * w0 : 0.f) + (w1 != 0.f ? o1[c] * w1 : 0.f);
+                }
             }
-        }
-        named_bar_sync(3, 256);
-        const int chunks = q_rows * (D / 8);
-        for (int idx = tid - W_SOFT0 * 32; idx < chunks; idx += 256) {
-            const int qq = idx / (D / 8);
-            const int c8 = idx - qq * (D / 8);
-            *reinterpret_cast<uint4*>(a.out + (static_cast<long long>(q_row0) + qq) * D + c8 * 8) =
-                *reinterpret_cast<const uint4*>(ostage + qq * D + c8 * 8);
+        } else {
+            if (t < D) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int cc = 32 * g + c;
+                    const float w0 = x.wgt[0][cc], w1 = x.wgt[1][cc];
+                    ostage[cc * D + t] = __float2bfloat16_rn((w0 != 0.f ? o0[c] * w0 : 0.f) + (w1 != 0.f ? o1[c] * w1 : 0.f));
+                }
+            }
+            named_bar_sync(3, 256);
+            const int chunks = q_rows * (D / 8);
+            for (int idx = tid - W_SOFT0 * 32; idx < chunks; idx += 256) {
+                const int qq = idx / (D / 8);
+                const int c8 = idx - qq * (D / 8);
+                *reinterpret_cast<uint4*>(a.out + (static_cast<long long>(q_row0) + qq) * D + c8 * 8) =
+                    *reinterpret_cast<const uint4*>(ostage + qq * D + c8 * 8);
+            }
         }
     }
 
@@ -575,6 +610,80 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (warp == W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// Merge of the list pieces of the query blocks past n_whole: with (M_p, L_p) the
+// max and denominator of piece p and O_p its normalised rows,
+//   out = sum_p 2^(M_p - M) L_p O_p / sum_p 2^(M_p - M) L_p,   M = max_p M_p,
+// the same softmax over the union of the pieces' keys. A warp per query row,
+// eight rows per CTA; lane l holds head-dim elements [V l, V l + V). Lane i
+// computes the weight of piece p0 + i, which a shuffle hands to the whole warp,
+// so the loads of consecutive pieces are independent.
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a)
+{
+    constexpr int V = D / 32;  // 4 (head_dim 128) or 2 (head_dim 64)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tr = blockIdx.x >> 3;                     // query block index past n_whole
+    const int qq = ((blockIdx.x & 7) << 3) + warp;      // row within the query block
+    const int row = a.n_whole + tr;
+    const int bh = row / a.Rq;
+    const int r = row - bh * a.Rq;
+    const int fq = r / a.bpf;
+    const int jq = r - fq * a.bpf;
+    const int q_rows = (jq == a.bpf - 1) ? a.rem : 64;
+    if (qq >= q_rows) return;
+    // launched as a programmatic dependent of the attention grid: wait until that
+    // grid has finished and its partial rows are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const long long q_row = static_cast<long long>(bh) * a.Lq + fq * a.F + jq * 64 + qq;
+    const long long s0 = static_cast<long long>(tr) * a.pieces;
+    const float* ml = a.part_ml + (s0 * 64 + qq) * 2;          // piece p at ml[p * 128]
+    const float* po = a.part_o + (s0 * 64 + qq) * D + V * lane;  // piece p at po[p * 64 * D]
+    float M = -INFINITY;
+    for (int p = lane; p < a.pieces; p += 32) M = fmaxf(M, ml[static_cast<long long>(p) * 128]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    float den = 0.f;
+    for (int p0 = 0; p0 < a.pieces; p0 += 32) {
+        float wl = 0.f;
+        if (p0 + lane < a.pieces) {
+            const float mp = ml[static_cast<long long>(p0 + lane) * 128];
+            if (mp != -INFINITY) wl = fast_exp2(mp - M) * ml[static_cast<long long>(p0 + lane) * 128 + 1];
+        }
+        den += wl;
+        const int np = min(32, a.pieces - p0);
+#pragma unroll 4
+        for (int i = 0; i < np; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+            const float* src = po + static_cast<long long>(p0 + i) * 64 * D;
+            if constexpr (V == 4) {
+                const float4 x = *reinterpret_cast<const float4*>(src);
+                acc[0] += w * x.x;
+                acc[1] += w * x.y;
+                acc[2] += w * x.z;
+                acc[3] += w * x.w;
+            } else {
+                const float2 x = *reinterpret_cast<const float2*>(src);
+                acc[0] += w * x.x;
+                acc[1] += w * x.y;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint16_t* out = a.out + q_row * D + V * lane;
+    if constexpr (V == 4) {
+        const uint32_t lo = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        const uint32_t hi = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(out) = make_uint2(lo, hi);
+    } else {
+        *reinterpret_cast<uint32_t*>(out) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
     }
 }
 
@@ -592,9 +701,23 @@ cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, int n_rows, cuda
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    attn_kernel<D, IL><<<static_cast<unsigned>(n_rows), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
-                                                                               m.v_rem, a);
-    return cudaGetLastError();
+    const int tail = a.pieces > 0 ? n_rows - a.n_whole : 0;
+    const long long grid = a.pieces > 0 ? a.n_whole + static_cast<long long>(tail) * a.pieces : n_rows;
+    attn_kernel<D, IL><<<static_cast<unsigned>(grid), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
+                                                                             m.v_rem, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || tail == 0) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tail) * 8u);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_merge_kernel<D>, a);
 }
 
 }  // namespace

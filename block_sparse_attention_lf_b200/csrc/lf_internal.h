@@ -45,6 +45,13 @@ struct AttnArgs {
     long long kv_stride;
     float scale_log2;  // softmax scale * log2(e)
     int* err;
+    // Split of the last, partial wave: query blocks [0, n_whole) take one CTA
+    // each; every later query block's list is cut into `pieces` consecutive
+    // pieces, one CTA each, whose normalised fp32 partial rows and (max, sum)
+    // pairs go to part_o / part_ml and are merged by a second kernel.
+    int n_whole, pieces;  // pieces == 0: no split
+    float* part_o;        // [slot][64][D]; slot = (query block - n_whole) * pieces + piece
+    float* part_ml;       // [slot][64][2]: max of scale*log2(e)*score, softmax denominator
 };
 
 struct AttnMaps {

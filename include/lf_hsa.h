@@ -16,6 +16,9 @@
  *                        written as a compacted block list (the mask B_r)
  *   lf_block_sparse_attn softmax attention of each query block over the valid
  *                        tokens of its listed KV blocks (tcgen05 tensor cores)
+ *   lf_block_sparse_attn_ws  the same with the last, partial wave of query
+ *                        blocks split into list pieces (caller workspace)
+ *   lf_attn_split_plan   that split's plan and workspace size (host only)
  *
  * plus the host-side Chunk-Aware Growth budget solver (same pages, stage 1 /
  * Technical Summary 2.1).
@@ -200,6 +203,48 @@ LF_API lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t*
                                const uint16_t* v, const int32_t* block_list,
                                const int32_t* block_count, int32_t list_cap, float softmax_scale,
                                uint16_t* out, void* stream);
+
+/*
+ * lf_block_sparse_attn with the last, partial wave split (same passage; the
+ * split is a scheduling choice and changes the result only by fp32 rounding).
+ * One CTA computes one query block; with n_rows = B*H*Rq query blocks on a
+ * device of sm SMs the last r = n_rows mod sm of them (all of them when
+ * n_rows < sm) would run alone on r SMs. Their lists are cut into `pieces`
+ * consecutive pieces, each piece's softmax partial (normalised rows plus the
+ * row max and denominator) goes to `workspace`, and a second kernel merges
+ * the pieces of each row exactly as the online softmax would.
+ *   tail_pieces      0: automatic plan (lf_attn_split_plan on the current
+ *                    device); 1: no split; >= 2: that many pieces per list.
+ *                    The piece count is lowered to what `workspace` holds and
+ *                    to list_cap; below 2 nothing is split.
+ *   workspace        device scratch, 16-byte aligned, owned by the caller,
+ *                    64 * (head_dim + 2) * 4 bytes per piece slot (r * pieces
+ *                    slots); NULL with workspace_bytes == 0 means no split.
+ *                    Two calls in flight at once need two workspaces.
+ * Enqueues two kernels when it splits, one otherwise.
+ * Errors: those of lf_block_sparse_attn; LF_ERR_ARG for tail_pieces < 0 or
+ * workspace_bytes < 0; LF_ERR_NULL / LF_ERR_ALIGN for the workspace.
+ */
+LF_API lf_status lf_block_sparse_attn_ws(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                                  const uint16_t* v, const int32_t* block_list,
+                                  const int32_t* block_count, int32_t list_cap, float softmax_scale,
+                                  uint16_t* out, int32_t tail_pieces, void* workspace,
+                                  int64_t workspace_bytes, void* stream);
+
+/*
+ * The automatic split plan of lf_block_sparse_attn_ws, host only.
+ *   sm               SM count to plan for; <= 0 queries the current device
+ *                    (LF_ERR_NO_DEVICE without one).
+ *   tail_rows out    query blocks whose lists are split (0: no split)
+ *   pieces out       pieces per split list: min(sm / tail_rows, list_cap / 8);
+ *                    0 (no split) when sm / tail_rows < 8 (the last wave
+ *                    fills more than an eighth of the SMs) or the minimum is
+ *                    below 2
+ *   workspace_bytes out  tail_rows * pieces * 64 * (head_dim + 2) * 4
+ * Errors: LF_ERR_NULL, LF_ERR_SHAPE, LF_ERR_CAP, LF_ERR_NO_DEVICE.
+ */
+LF_API lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap, int32_t sm,
+                             int32_t* tail_rows, int32_t* pieces, int64_t* workspace_bytes);
 
 /*
  * Chunk-Aware Growth budget solver, host only, fp64 (paper.rainbus.top,

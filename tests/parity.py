@@ -30,13 +30,14 @@ OUT_REL_FRO = 1e-2
 
 
 def run_gpu(shape, q, k, v, chunk: int, kf: int, kb: int, scale: float = 0.0,
-            kv_stride: int = 0) -> Dict[str, np.ndarray]:
-    """Run the four device steps through the C ABI; returns host copies."""
+            kv_stride: int = 0, tail_pieces: int = 0) -> Dict[str, np.ndarray]:
+    """Run the four device steps through the C ABI; returns host copies.
+    ``tail_pieces`` as in ``HSACall`` (0: the automatic split of the last wave)."""
     import block_sparse_attention_lf_b200 as L
     s = L.LfShape.make(shape.batch, shape.heads, shape.head_dim, shape.frame_tokens,
                        shape.n_frames, shape.n_sink, shape.n_recent, shape.n_cur,
                        kv_stride=kv_stride)
-    call = L.HSACall(s, chunk, kf, kb, softmax_scale=scale)
+    call = L.HSACall(s, chunk, kf, kb, softmax_scale=scale, tail_pieces=tail_pieces)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     call(qd, kd, vd)
     torch.cuda.synchronize()
@@ -46,7 +47,8 @@ def run_gpu(shape, q, k, v, chunk: int, kf: int, kb: int, scale: float = 0.0,
     return dict(q_pool=b.q_pool.cpu().double().numpy(), k_pool=b.k_pool.cpu().double().numpy(),
                 k_frame=b.k_frame.cpu().double().numpy(), frame_sel=b.frame_sel.cpu().numpy(),
                 block_list=b.block_list.cpu().numpy(), block_count=b.block_count.cpu().numpy(),
-                out=b.out.cpu().float().numpy().astype(np.float64), list_cap=b.list_cap)
+                out=b.out.cpu().float().numpy().astype(np.float64), list_cap=b.list_cap,
+                split=call.split)
 
 
 def check_pool(g: dict, o: dict, q, k) -> None:

@@ -173,3 +173,57 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         L.lf_pool(sh, q, q, q.float(), q.float(), q.float())
+
+
+def test_attn_ws_validation():
+    sh = _shape()
+    p = ctypes.c_void_p(FAKE)
+    mis = ctypes.c_void_p(FAKE + 8)
+    S = ctypes.byref(sh)
+    f = L.lib.lf_block_sparse_attn_ws
+    assert f(ctypes.byref(_shape(head_dim=96)), p, p, p, p, p, 108, 0.0, p, 0, p, 1 << 20, None) == 3
+    assert f(S, p, p, p, p, p, -1, 0.0, p, 0, p, 1 << 20, None) == 5
+    assert f(S, p, p, p, p, p, 108, 0.0, p, -1, p, 1 << 20, None) == 9   # tail_pieces < 0
+    assert f(S, p, p, p, p, p, 108, 0.0, p, 0, p, -16, None) == 9        # workspace_bytes < 0
+    assert f(S, p, p, p, p, p, 108, 0.0, p, 0, None, 1 << 20, None) == 1  # bytes without a workspace
+    assert f(S, p, p, p, p, p, 108, 0.0, p, 0, mis, 1 << 20, None) == 2
+    assert f(S, p, p, None, p, p, 108, 0.0, p, 0, p, 1 << 20, None) == 1
+
+
+def _plan_rule(n_rows, sm, cap):
+    """The split rule as the header states it."""
+    r = n_rows % sm
+    if r == 0 or sm // r < 8:
+        return 0, 0
+    k = min(sm // r, cap // 8, cap)
+    return (r, k) if k >= 2 else (0, 0)
+
+
+@pytest.mark.parametrize("B,H,nc,kb,sm", [
+    (1, 12, 3, 12, 148),   # 900 query blocks: 12 in the last wave, lists of 108
+    (2, 12, 3, 12, 148),   # 1800: 24 in the last wave
+    (1, 2, 3, 12, 148),    # 150: 2 left over
+    (1, 1, 1, 12, 148),    # fewer query blocks than SMs: every list split
+    (1, 12, 3, 1, 148),    # lists of 9 entries: pieces capped at 9 // 8 = 1, no split
+    (1, 4, 37, 12, 148),   # 4 * 37 * 25 = 3700 = 25 waves of 148: no tail
+    (1, 12, 3, 12, 132),   # another SM count
+    (1, 24, 3, 12, 148),   # 1800 = 12 waves + 24: the last wave fills 16 % of the SMs, no split
+])
+def test_split_plan(B, H, nc, kb, sm):
+    sh = L.LfShape.make(B, H, 128, 1560, 18 + nc, 1, 1, nc)
+    cap = L.lf_list_capacity(sh, 2, 4, kb)
+    t, k, nbytes = L.lf_attn_split_plan(sh, cap, sm)
+    n_rows = B * H * sh.Rq
+    assert (t, k) == _plan_rule(n_rows, sm, cap)
+    assert nbytes == t * k * 64 * (128 + 2) * 4
+    if (B, H, nc, kb, sm) == (1, 12, 3, 12, 148):
+        assert (t, k) == (12, 12)
+
+
+def test_split_plan_validation():
+    sh = _shape()
+    t, k, b = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int64()
+    f = L.lib.lf_attn_split_plan
+    assert f(ctypes.byref(sh), -1, 148, ctypes.byref(t), ctypes.byref(k), ctypes.byref(b)) == 5
+    assert f(ctypes.byref(sh), 108, 148, None, ctypes.byref(k), ctypes.byref(b)) == 1
+    assert f(ctypes.byref(_shape(head_dim=96)), 108, 148, ctypes.byref(t), ctypes.byref(k), ctypes.byref(b)) == 3

@@ -31,8 +31,8 @@ def _rand(seed, B, H, Lq, Lkv, D, kscale=1.0, kv_stride=0):
     return q, k, v
 
 
-def _full_check(shape, q, k, v, chunk, kf, kb, kv_stride=0, rows=None):
-    g = parity.run_gpu(shape, q, k, v, chunk, kf, kb, kv_stride=kv_stride)
+def _full_check(shape, q, k, v, chunk, kf, kb, kv_stride=0, rows=None, tail_pieces=0):
+    g = parity.run_gpu(shape, q, k, v, chunk, kf, kb, kv_stride=kv_stride, tail_pieces=tail_pieces)
     s_or = oracle.Shape(shape.batch, shape.heads, shape.head_dim, shape.frame_tokens, 64,
                         shape.n_frames, shape.n_sink, shape.n_recent, shape.n_cur, kv_stride=kv_stride)
     qp, kp, kfr = oracle.pool(s_or, q, k)
@@ -79,6 +79,24 @@ def test_tiny_workload_full():
     assert fr["exact"] > 0
 
 
+def _tail_rows(shape, chunk, kf, kb):
+    """First and last valid token rows of every query block whose list the automatic plan
+    splits (the last, partial wave of one-CTA-per-query-block attention)."""
+    import block_sparse_attention_lf_b200 as L
+    s = L.LfShape.make(shape.batch, shape.heads, shape.head_dim, shape.frame_tokens, shape.n_frames,
+                       shape.n_sink, shape.n_recent, shape.n_cur)
+    tail, pieces, _ = L.lf_attn_split_plan(s, L.lf_list_capacity(s, chunk, kf, kb))
+    n_rows = shape.batch * shape.heads * shape.Rq
+    out = []
+    for qb in range(n_rows - tail, n_rows):
+        bh, r = divmod(qb, shape.Rq)
+        f, j = divmod(r, shape.bpf)
+        t0 = f * shape.frame_tokens + j * 64
+        t1 = min(t0 + 64, (f + 1) * shape.frame_tokens) - 1
+        out += [bh * shape.Lq + t0, bh * shape.Lq + t1]
+    return np.array(out, dtype=np.int64)
+
+
 def _kb(w, shape):
     if w.topk_blocks:
         return w.topk_blocks
@@ -94,6 +112,7 @@ def test_full_size_workloads(name, kb_override):
     shape = oracle.shape_of(w)
     kb = kb_override or _kb(w, shape)
     rows = parity.sample_rows(shape, per_block=3, blocks_per_head=5, seed=1)
+    rows = np.union1d(rows, _tail_rows(shape, w.chunk_index, w.topk_frames, kb))
     fr, bl, at = _full_check(shape, q, k, v, w.chunk_index, w.topk_frames, kb, rows=rows)
     # the planted structure makes most frame cuts clear
     assert fr["exact"] >= 0.5 * (fr["exact"] + fr["tie"])
@@ -149,3 +168,45 @@ def test_pool_range_reuses_past_frames():
     L.lf_pool_range(ls, qd, kd, 3, 3, qp, kp, kfr, pool_q=False)
     torch.cuda.synchronize()
     assert torch.equal(before, kp)
+
+
+SPLIT = [("ragged_d128", 2), ("ragged_d64_odd_lists", 3), ("kv_head_stride", 2),
+         ("all_keep", 5), ("sharp_softmax_rescales", 4), ("long_lists_many_tiles", 7),
+         ("long_lists_many_tiles", 1000)]
+
+
+@pytest.mark.parametrize("name,pieces", SPLIT, ids=[f"{n}-{p}" for n, p in SPLIT])
+def test_small_cases_split(name, pieces):
+    """Every list cut into `pieces` pieces (fewer query blocks than SMs: all of them are in the
+    last wave); 1000 pieces leaves most pieces empty (the count is capped at the list length)."""
+    case = next(c for c in SMALL if c[0] == name)
+    _, B, H, D, F, (ns, nm, nr, nc), chunk, kf, kb, kscale, pad = case
+    NF = ns + nm + nr + nc
+    shape = oracle.Shape(B, H, D, F, 64, NF, ns, nr, nc)
+    stride = NF * F + pad if pad else 0
+    q, k, v = _rand(zlib.crc32(name.encode()) % 1000, B, H, nc * F, NF * F, D, kscale, stride)
+    g = parity.run_gpu(shape, q, k, v, chunk, kf, kb, kv_stride=stride, tail_pieces=pieces)
+    assert g["split"][0] == B * H * shape.Rq and g["split"][1] >= 2
+    s_or = oracle.Shape(B, H, D, F, 64, NF, ns, nr, nc, kv_stride=stride)
+    parity.check_attention(s_or, q, k, v, g)
+
+
+def test_split_matches_unsplit_layer480p():
+    """The automatic split changes only the last wave's query blocks, and those only by rounding."""
+    w = lf_synth.CONFIGS["layer480p"]
+    q, k, v = lf_synth.make_qkv(w)
+    shape = oracle.shape_of(w)
+    kb = _kb(w, shape)
+    a = parity.run_gpu(shape, q, k, v, w.chunk_index, w.topk_frames, kb, tail_pieces=1)
+    b = parity.run_gpu(shape, q, k, v, w.chunk_index, w.topk_frames, kb)
+    tail, pieces = b["split"]
+    assert a["split"] == (0, 0) and tail > 0 and pieces >= 2
+    np.testing.assert_array_equal(a["block_list"], b["block_list"])
+    oa, ob = a["out"].reshape(-1, shape.head_dim), b["out"].reshape(-1, shape.head_dim)
+    n_rows = shape.batch * shape.heads * shape.Rq
+    bh0, r0 = divmod(n_rows - tail, shape.Rq)
+    f0, j0 = divmod(r0, shape.bpf)
+    first_tail_row = bh0 * shape.Lq + f0 * shape.frame_tokens + j0 * 64
+    np.testing.assert_array_equal(oa[:first_tail_row], ob[:first_tail_row])
+    d = np.abs(oa[first_tail_row:] - ob[first_tail_row:]).max()
+    assert d <= parity.OUT_MAX_ABS, d
