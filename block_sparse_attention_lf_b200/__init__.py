@@ -34,15 +34,15 @@ __all__ = [
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
     "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
-    "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
-    "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
+    "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_block_sparse_attn_static",
+    "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
 )
 
 LF_OK = 0
 STATUS_NAMES = {
     0: "LF_OK", 1: "LF_ERR_NULL", 2: "LF_ERR_ALIGN", 3: "LF_ERR_SHAPE", 4: "LF_ERR_TOPK",
     5: "LF_ERR_CAP", 6: "LF_ERR_INFEASIBLE", 7: "LF_ERR_CUDA", 8: "LF_ERR_DEVICE_TIMEOUT",
-    9: "LF_ERR_ARG", 10: "LF_ERR_LIST", 11: "LF_ERR_NO_DEVICE",
+    9: "LF_ERR_ARG", 10: "LF_ERR_LIST", 11: "LF_ERR_NO_DEVICE", 12: "LF_ERR_SCRATCH",
 }
 
 
@@ -108,6 +108,7 @@ def _load() -> ctypes.CDLL:
         "lf_block_sparse_attn_ws": ([S, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
         "lf_attn_split_plan": ([S, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
                                 ctypes.POINTER(ctypes.c_int64)], I32),
+        "lf_block_sparse_attn_static": ([S, P, P, P, P, P, I32, F32, P, I32, P], I32),
         "lf_cag_budget": ([I32, P, P, F64, F64, I32, P, P], I32),
         "lf_blocks_for_sparsity": ([F64, I32, I32, I32], I32),
         "lf_get_device_error": ([ctypes.POINTER(I32)], I32),

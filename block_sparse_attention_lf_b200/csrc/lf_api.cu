@@ -203,6 +203,7 @@ const char* lf_status_string(lf_status s)
     case LF_ERR_ARG: return "invalid argument";
     case LF_ERR_LIST: return "block id or count out of range";
     case LF_ERR_NO_DEVICE: return "no usable CUDA device";
+    case LF_ERR_SCRATCH: return "the call needs more than the library's static scratch array";
     }
     return "unknown status";
 }
@@ -415,3 +416,58 @@ lf_status lf_get_device_error(int32_t* detail)
 }
 
 }  // extern "C"
+
+// ---- attention without allocation ---------------------------------------------
+// The split's partial rows for lf_block_sparse_attn_static: a fixed array in the
+// library image, so that callers that cannot allocate device memory need not.
+static __device__ __align__(256) unsigned char g_attn_scratch[LF_ATTN_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_attn_scratch on the current device (looked up once per
+// device; host code cannot use the symbol itself as a device pointer).
+lf_status static_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return LF_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return LF_OK;
+}
+
+}  // namespace
+
+extern "C" lf_status lf_block_sparse_attn_static(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                                                const uint16_t* v, const int32_t* block_list,
+                                                const int32_t* block_count, int32_t list_cap,
+                                                float softmax_scale, uint16_t* out, int32_t tail_pieces,
+                                                void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (list_cap < 0) return LF_ERR_CAP;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale) || tail_pieces < 0) return LF_ERR_ARG;
+    if (!q || !k || !v || !block_list || !block_count || !out) return LF_ERR_NULL;
+    // scratch the split needs: the same plan lf_block_sparse_attn_ws makes
+    long long need = 0;
+    if (tail_pieces != 1) {
+        int sm = 0;
+        if ((st = sm_count(&sm)) != LF_OK) return st;
+        int t = 0, kp = 0;
+        split_plan(static_cast<long long>(d.B) * d.H * d.Rq, sm, list_cap, tail_pieces, -1, &t, &kp);
+        need = static_cast<long long>(t) * kp * split_slot_bytes(d.D);
+    }
+    if (need > LF_ATTN_STATIC_SCRATCH_BYTES) return LF_ERR_SCRATCH;
+    void* ws = nullptr;
+    if (need > 0 && (st = static_scratch(&ws)) != LF_OK) return st;
+    return lf_block_sparse_attn_ws(shape, q, k, v, block_list, block_count, list_cap, softmax_scale, out,
+                                   need > 0 ? tail_pieces : 1, ws, need, stream);
+}

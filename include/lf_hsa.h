@@ -76,7 +76,8 @@ typedef enum lf_status {
     LF_ERR_DEVICE_TIMEOUT = 8, /* device error word: a bounded wait in a kernel expired */
     LF_ERR_ARG = 9,            /* another invalid scalar (chunk index, sparsity, scale) */
     LF_ERR_LIST = 10,          /* device error word: a block id or count out of range */
-    LF_ERR_NO_DEVICE = 11      /* no usable sm_100 device */
+    LF_ERR_NO_DEVICE = 11,     /* no usable sm_100 device */
+    LF_ERR_SCRATCH = 12        /* the call needs more than the library's static scratch array */
 } lf_status;
 
 /*
@@ -245,6 +246,40 @@ LF_API lf_status lf_block_sparse_attn_ws(const lf_hsa_shape* shape, const uint16
  */
 LF_API lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap, int32_t sm,
                              int32_t* tail_rows, int32_t* pieces, int64_t* workspace_bytes);
+
+/* Size of the scratch array behind lf_block_sparse_attn_static. */
+#define LF_ATTN_STATIC_SCRATCH_BYTES (8ll << 20)
+
+/*
+ * lf_block_sparse_attn_ws for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a packaging of the same computation.
+ * Some callers have no way to allocate: a plug-in inside a host application
+ * that owns the whole device-memory budget and hands out no allocator, or a
+ * loop that must not call cudaMalloc / cudaFree because they synchronise the
+ * device and may fail once the budget is spent. Such a caller passes only its
+ * inputs and outputs; the split's partial rows go to a scratch array of
+ * LF_ATTN_STATIC_SCRATCH_BYTES (8 MiB) compiled into this library, which every
+ * GPU that loads the library holds until the process exits. The call
+ * allocates nothing.
+ *   tail_pieces  as in lf_block_sparse_attn_ws (0: automatic plan, 1: no
+ *                split, >= 2: that many pieces per split list).
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ * first call before any stream capture.
+ * Sharing: every call on a device uses the same array and leaves its partial
+ * rows in it. Each call writes every slot it reads before reading it, so
+ * nothing has to start at zero, but two calls that overlap on the GPU (other
+ * streams, other threads) race on the array and give wrong results: order them.
+ * Errors: those of lf_block_sparse_attn_ws; LF_ERR_SCRATCH (nothing launched)
+ * when the split would need more than LF_ATTN_STATIC_SCRATCH_BYTES, i.e. more
+ * than LF_ATTN_STATIC_SCRATCH_BYTES / (64 * (head_dim + 2) * 4) piece slots
+ * (the automatic plan uses at most one slot per SM: 148 of 252 at head_dim 128).
+ */
+LF_API lf_status lf_block_sparse_attn_static(const lf_hsa_shape* shape, const uint16_t* q, const uint16_t* k,
+                                      const uint16_t* v, const int32_t* block_list,
+                                      const int32_t* block_count, int32_t list_cap,
+                                      float softmax_scale, uint16_t* out, int32_t tail_pieces,
+                                      void* stream);
 
 /*
  * Chunk-Aware Growth budget solver, host only, fp64 (paper.rainbus.top,
