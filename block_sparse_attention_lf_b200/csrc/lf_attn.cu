@@ -53,6 +53,13 @@
 //     flag and the device error word, every role runs its remaining steps
 //     without waiting, in-flight copies and MMAs are drained, TMEM is freed,
 //     and the kernel returns.
+//   * Split of the last wave (optional, AttnArgs::pieces > 0): query blocks
+//     past n_whole would run as a last, partial wave on a few SMs, so each of
+//     their lists is cut into `pieces` consecutive pieces, one CTA each. Such
+//     a CTA runs the same code on its sub-list and ends by writing normalised
+//     fp32 rows and each row's (max, denominator) instead of bf16 output;
+//     attn_merge_kernel then combines the pieces of each row the way the
+//     online softmax would.
 #include "lf_device.cuh"
 #include "lf_internal.h"
 
