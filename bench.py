@@ -3,7 +3,8 @@
 
 A step is one whole HSA call on resident inputs: block/frame mean pooling,
 frame selection, block selection and block-sparse attention (four kernels of
-liblf_hsa.so, called through the C ABI). The default workload is the
+liblf_hsa.so, called through the C ABI, plus the merge kernel when the
+attention splits the lists of its last, partial wave). The default workload is the
 480p-shaped layer call (batch 1, 12 heads, head_dim 128, 1560-token frames,
 21 KV frames = sink + 16 memory + recent + 3-frame current chunk, frame top-4,
 block top-k for 80 % block sparsity), drawn by ``lf_synth``.
