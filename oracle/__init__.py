@@ -49,6 +49,8 @@ def configure(lib):
     lib.orc_select_frames.restype = None
     lib.orc_select_blocks.argtypes = [_i] * 9 + [_p, _p, _p, _p, _p, _i, _p]
     lib.orc_select_blocks.restype = _i
+    lib.orc_select_blocks_1d.argtypes = [_i] * 7 + [_p, _p, _p, _p, _i, _p]
+    lib.orc_select_blocks_1d.restype = _i
     lib.orc_attention.argtypes = [_i] * 6 + [_l, _p, _p, _p, _p, _p, _i, _d, _p, _l, _p]
     lib.orc_attention.restype = None
     lib.orc_cag.argtypes = [_i, _p, _p, _d, _d, _i, _p, _p]
@@ -175,6 +177,26 @@ def select_blocks(s: Shape, chunk_index: int, topk_blocks: int, q_pool: np.ndarr
     rc = lib.orc_select_blocks(s.batch, s.heads, s.head_dim, s.Rq, s.n_frames, s.bpf, n_sel,
                                chunk_index, topk_blocks, _ptr(qp), _ptr(kp), _ptr(fs), _ptr(lst),
                                _ptr(cnt), cap, _ptr(sc))
+    if rc != 0:
+        raise ValueError("block list exceeds list_cap")
+    return lst, cnt, sc
+
+
+def select_blocks_1d(s: Shape, chunk_index: int, topk_blocks: int, q_pool: np.ndarray,
+                     k_pool: np.ndarray, list_cap: Optional[int] = None
+                     ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """One-dimensional selection (global block top-k, no frame level):
+    (block_list [B,H,Rq,cap], block_count [B,H,Rq], block scores [B,H,Rq,Nkv])."""
+    lib = _load()
+    keep = s.Nkv if (chunk_index == 1 or topk_blocks > s.Nkv) else topk_blocks
+    cap = list_cap if list_cap is not None else keep
+    qp = np.ascontiguousarray(q_pool, np.float64)
+    kp = np.ascontiguousarray(k_pool, np.float64)
+    lst = np.full((s.batch, s.heads, s.Rq, cap), -1, np.int32)
+    cnt = np.zeros((s.batch, s.heads, s.Rq), np.int32)
+    sc = np.zeros((s.batch, s.heads, s.Rq, s.Nkv), np.float64)
+    rc = lib.orc_select_blocks_1d(s.batch, s.heads, s.head_dim, s.Rq, s.Nkv, chunk_index, topk_blocks,
+                                  _ptr(qp), _ptr(kp), _ptr(lst), _ptr(cnt), cap, _ptr(sc))
     if rc != 0:
         raise ValueError("block list exceeds list_cap")
     return lst, cnt, sc

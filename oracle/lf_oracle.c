@@ -30,7 +30,8 @@
  * forced ones included; selection is per (batch, head, query block); scores are
  * plain inner products; attention uses scale/softmax over exactly the valid
  * tokens of the kept blocks with no causal mask; a query block with an empty
- * list gets a zero output.
+ * list gets a zero output; the one-dimensional ablation variant is a global
+ * block top-k with no frame level and no forced frames.
  *
  * Inputs q, k, v are bf16 bit patterns (uint16). Step 1 of every routine converts
  * them to fp64 exactly; all arithmetic after that is fp64.
@@ -229,6 +230,46 @@ int orc_select_blocks(int B, int H, int D, int Rq, int NF, int bpf, int n_sel,
             block_count[bh * Rq + r] = n;
         }
     free(row);
+    free(cand);
+    return rc;
+}
+
+/*
+ * One-dimensional ("1-D") block selection: the single-granularity sparse
+ * attention of the ablation in [NE] section 4 (one-dimensional sparse attention
+ * without the frame level). Reading (the pages name the variant but do not
+ * spell it out): every KV block g of every frame is a candidate,
+ * o_r(g) = <q~_r, k~_g>, and the mask row keeps the top-k of them (ties to the
+ * lower index) with no frame forced in. The row is written as ascending block
+ * ids with its length in block_count. chunk_index == 1 keeps every block (dense
+ * first chunk, [RB] stage 1). If block_scores is not NULL it receives o_r(g) as
+ * [B,H,Rq,Nkv]. Returns 0, or -1 if a row would exceed list_cap.
+ */
+int orc_select_blocks_1d(int B, int H, int D, int Rq, int Nkv, int chunk_index, int topk_blocks,
+                         const double* q_pool, const double* k_pool,
+                         int* block_list, int* block_count, int list_cap, double* block_scores)
+{
+    int keep = (chunk_index == 1 || topk_blocks > Nkv) ? Nkv : topk_blocks;
+    scored* cand = (scored*)malloc(sizeof(scored) * (size_t)(Nkv > 0 ? Nkv : 1));
+    int* kept = (int*)malloc(sizeof(int) * (size_t)(Nkv > 0 ? Nkv : 1));
+    int rc = 0;
+    for (long bh = 0; bh < (long)B * H; ++bh)
+        for (int r = 0; r < Rq; ++r) {
+            const double* qr = q_pool + (bh * Rq + r) * (long)D;
+            for (int g = 0; g < Nkv; ++g) {
+                cand[g].idx = g;
+                cand[g].score = dot(qr, k_pool + (bh * (long)Nkv + g) * D, D);
+                if (block_scores) block_scores[(bh * Rq + r) * (long)Nkv + g] = cand[g].score;
+            }
+            qsort(cand, (size_t)Nkv, sizeof(scored), by_score_then_index);
+            for (int t = 0; t < keep; ++t) kept[t] = cand[t].idx;
+            qsort(kept, (size_t)keep, sizeof(int), by_int);
+            int n = keep;
+            if (n > list_cap) { rc = -1; n = list_cap; }
+            memcpy(block_list + (bh * Rq + r) * (long)list_cap, kept, sizeof(int) * (size_t)n);
+            block_count[bh * Rq + r] = n;
+        }
+    free(kept);
     free(cand);
     return rc;
 }

@@ -26,6 +26,10 @@ PINS = [
     t_sel.test_select_hand_worked,
     lambda: [t_sel.test_select_brute_force_with_ties(s) for s in range(6)],
     lambda: [t_sel.test_select_invariants(*a) for a in [(2, 2, 2), (2, 9, 3), (2, 1, 99), (1, 2, 2)]],
+    lambda: [t_sel.test_select_1d_brute_force_with_ties(s) for s in range(6)],
+    lambda: [t_sel.test_select_1d_invariants(*a) for a in [(2, 1), (2, 7), (2, 10**6), (1, 3)]],
+    t_sel.test_select_1d_forces_no_frame,
+    t_sel.test_select_1d_matches_two_level_on_frame_structured_scores,
     lambda: [t_attn.test_all_keep_equals_dense_sdpa(*a) for a in [(100, 64, 16), (64, 64, 8)]],
     t_attn.test_single_block_and_partial_block,
     t_attn.test_rows_subset_and_empty_list,
@@ -54,6 +58,10 @@ MUTATIONS = [
     ("CAG sign flipped", "s_out[i] = s_base - beta / sqrt(T[i]);", "s_out[i] = s_base + beta / sqrt(T[i]);"),
     ("CAG alpha = 1/T", "double alpha = 1.0 / sqrt(T[i]);", "double alpha = 1.0 / T[i];"),
     ("CAG dense chunk weight dropped", "if (target_over_all) W += w[i];", ""),
+    ("1-D keeps one block too few", "for (int t = 0; t < keep; ++t) kept[t] = cand[t].idx;", "for (int t = 0; t + 1 < keep; ++t) kept[t] = cand[t].idx;"),
+    ("1-D scores the neighbouring block", "cand[g].score = dot(qr, k_pool + (bh * (long)Nkv + g) * D, D);", "cand[g].score = dot(qr, k_pool + (bh * (long)Nkv + (g + 1) % Nkv) * D, D);"),
+    ("1-D list left in score order", "qsort(kept, (size_t)keep, sizeof(int), by_int);", ""),
+    ("1-D first chunk not dense", "int keep = (chunk_index == 1 || topk_blocks > Nkv) ? Nkv : topk_blocks;", "int keep = topk_blocks > Nkv ? Nkv : topk_blocks;"),
     ("k_b truncates instead of rounding", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel);"),
 ]
 

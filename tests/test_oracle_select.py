@@ -122,3 +122,86 @@ def test_select_invariants(chunk_index, kf, kb):
         assert {g // s.bpf for g in blocks} == set(r_sel.tolist())
     if chunk_index == 1:
         assert (lst == np.arange(s.Nkv)).all()
+
+
+# ---- one-dimensional selection (the ablation's single-granularity variant) ----------
+# 163.com article, section 4 (ablation: one-dimensional sparse attention, no frame
+# level). Reading: a global top-k over all KV blocks, no forced frames, ties to the
+# lower index, ascending ids; the first chunk stays dense.
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_1d_brute_force_with_ties(seed):
+    """Integer pooled vectors (many exact ties) against the subset-enumeration top-k over
+    every KV block of every frame."""
+    rng = np.random.default_rng(100 + seed)
+    B, H, D = 1, 2, 3
+    s = oracle.Shape(B, H, D, 150, 64, 4, 1, 1, 1)  # 4 frames x 3 blocks = 12 candidates
+    q_pool = rng.integers(-2, 3, size=(B, H, s.Rq, D)).astype(np.float64)
+    k_pool = rng.integers(-2, 3, size=(B, H, s.Nkv, D)).astype(np.float64)
+    kb = 1 + seed
+    lst, cnt, sc = oracle.select_blocks_1d(s, 2, kb, q_pool, k_pool)
+    for b in range(B):
+        for h in range(H):
+            for r in range(s.Rq):
+                scores = [float(q_pool[b, h, r] @ k_pool[b, h, g]) for g in range(s.Nkv)]
+                np.testing.assert_array_equal(sc[b, h, r], scores)
+                expect = sorted(_topk_by_definition(scores, kb))
+                assert cnt[b, h, r] == len(expect)
+                assert lst[b, h, r, :cnt[b, h, r]].tolist() == expect
+
+
+@pytest.mark.parametrize("chunk_index,kb", [(2, 1), (2, 7), (2, 10**6), (1, 3)])
+def test_select_1d_invariants(chunk_index, kb):
+    """Every row keeps min(k, Nkv) blocks (all of them in the dense first chunk), as an
+    ascending list of distinct valid ids; no frame is forced in."""
+    rng = np.random.default_rng(12)
+    B, H, D = 2, 2, 8
+    s = oracle.Shape(B, H, D, 200, 64, 10, 2, 1, 2)
+    q_pool = rng.standard_normal((B, H, s.Rq, D))
+    k_pool = rng.standard_normal((B, H, s.Nkv, D))
+    lst, cnt, _ = oracle.select_blocks_1d(s, chunk_index, kb, q_pool, k_pool)
+    keep = s.Nkv if chunk_index == 1 else min(kb, s.Nkv)
+    assert (cnt == keep).all()
+    for r_lst, c in zip(lst.reshape(-1, lst.shape[-1]), cnt.reshape(-1)):
+        blocks = r_lst[:c].tolist()
+        assert blocks == sorted(set(blocks)) and 0 <= blocks[0] and blocks[-1] < s.Nkv
+    if chunk_index == 1:
+        assert (lst == np.arange(s.Nkv)).all()
+
+
+def test_select_1d_forces_no_frame():
+    """Sink blocks that score below every other block are never kept by the one-dimensional
+    selection, while the two-level selection always keeps the sink frame."""
+    rng = np.random.default_rng(14)
+    B, H, D = 1, 2, 4
+    s = oracle.Shape(B, H, D, 200, 64, 8, 1, 1, 2)
+    q_pool = np.abs(rng.standard_normal((B, H, s.Rq, D))) + 0.1
+    k_pool = np.abs(rng.standard_normal((B, H, s.Nkv, D))) + 0.1
+    k_pool[:, :, :s.bpf * s.n_sink] = -1.0  # every sink block scores below zero
+    lst, cnt, _ = oracle.select_blocks_1d(s, 2, s.Nkv - s.bpf * s.n_sink, q_pool, k_pool)
+    assert (lst >= s.bpf * s.n_sink).all()
+    k_frame = np.abs(rng.standard_normal((B, H, s.n_frames, D)))
+    sel, _ = oracle.select_frames(s, 2, 1, q_pool, k_frame)
+    assert (sel[..., 0] == 0).all()
+
+
+def test_select_1d_matches_two_level_on_frame_structured_scores():
+    """When every frame holds exactly k_b blocks that outscore every other block of every
+    frame, the global top-(frames * k_b) is the two-level selection with all frames kept and
+    top-k_b blocks per frame."""
+    rng = np.random.default_rng(13)
+    B, H, D, kb = 1, 2, 4, 2
+    s = oracle.Shape(B, H, D, 300, 64, 6, 1, 1, 1)  # bpf 5, 3 memory frames
+    q_pool = np.zeros((B, H, s.Rq, D))
+    q_pool[..., 0] = 1.0
+    k_pool = rng.standard_normal((B, H, s.Nkv, D)) * 0.1
+    k_frame = rng.standard_normal((B, H, s.n_frames, D))
+    for h in range(H):
+        for tau in range(s.n_frames):
+            hi = rng.choice(s.bpf, kb, replace=False)
+            k_pool[0, h, tau * s.bpf + hi, 0] += 10.0 + rng.random(kb)
+    sel, _ = oracle.select_frames(s, 2, s.n_mem, q_pool, k_frame)  # every frame kept
+    lst2, cnt2, _ = oracle.select_blocks(s, 2, kb, q_pool, k_pool, sel)
+    lst1, cnt1, _ = oracle.select_blocks_1d(s, 2, s.n_frames * kb, q_pool, k_pool)
+    np.testing.assert_array_equal(cnt1, cnt2)
+    np.testing.assert_array_equal(lst1, lst2)
