@@ -399,6 +399,59 @@ def config_report(L, lf_synth, peaks, steps, flush):
     return out
 
 
+def one_dim_report(L, lf_synth, peaks, steps, flush):
+    """layer480p with the one-dimensional selection (global block top-k over all
+    KV blocks, no frame level; the ablation's variant) at the two-level call's
+    kept-block budget: pooling, lf_select_blocks_1d and the attention."""
+    import torch
+    w = lf_synth.CONFIGS["layer480p"]
+    shape = L.shape_from_workload(w)
+    n_sel = L.lf_frames_selected(shape, w.chunk_index, w.topk_frames)
+    kb2 = _kb(L, shape, w)
+    keep = n_sel * kb2
+    q, k, v = (t.cuda() for t in lf_synth.make_qkv(w))
+    call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb2)
+    b = call.buf
+    if b.list_cap < keep:
+        raise RuntimeError("list capacity below the kept count")
+
+    def select():
+        L.lf_select_blocks_1d(shape, w.chunk_index, keep, b.q_pool, b.k_pool, b.block_list, b.block_count,
+                              b.list_cap)
+    for _ in range(3):
+        call.pool(q, k)
+        select()
+        call.attend(q, k, v)
+    torch.cuda.synchronize()
+    flops = credited_flops(b.block_list.cpu().numpy(), b.block_count.cpu().numpy(), shape.frame_tokens,
+                           shape.bpf, shape.head_dim, shape.n_cur)
+    stream = torch.cuda.current_stream()
+    E = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        e = E[i]
+        e[0].record(stream)
+        call.pool(q, k)
+        e[1].record(stream)
+        select()
+        e[2].record(stream)
+        call.attend(q, k, v)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    st, detail = L.lf_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error: {st} {detail:#x}")
+
+    def us(i0, i1):
+        return statistics.mean(E[j][i0].elapsed_time(E[j][i1]) * 1e3 for j in range(steps))
+    t, att = us(0, 3), us(2, 3)
+    return {"us_per_call": round(t, 2),
+            "kernels_us": {"pool": round(us(0, 1), 2), "select_1d": round(us(1, 2), 2), "attn": round(att, 2)},
+            "kept_blocks_per_row": keep, "kept_tflop": round(flops / 1e12, 5),
+            "tflops_call": round(flops / (t * 1e-6) / 1e12, 1),
+            "attn_frac_of_bf16_peak": round(flops / (att * 1e-6) / 1e12 / peaks["bf16"], 4)}
+
+
 def run_ours(a):
     import numpy as np
     import torch
@@ -530,6 +583,10 @@ def run_ours(a):
             "pooled keys of past frames kept from a first full pooling; each call re-pools the "
             "current chunk's frames and the queries (lf_pool_range)"))
         line["configs"] = config_report(L, lf_synth, peaks, a.config_steps, flush)
+        try:
+            line["configs"]["layer480p_1d"] = one_dim_report(L, lf_synth, peaks, a.config_steps, flush)
+        except Exception as e:  # an extra report never costs the main line
+            line["configs"]["layer480p_1d"] = {"error": repr(e)[:200]}
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         r = _oracle_sample(w, a.cpu_budget_s, q_h, k_h, v_h)
         line["cpu_baseline"] = {"value": r["flops"] / r["t_call"] / 1e12, "unit": "TFLOP/s",

@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "liblf_hsa.so")
 
 __all__ = [
     "LfShape", "LfError", "lib", "lf_pool", "lf_pool_range", "lf_select_frames", "lf_select_blocks",
+    "lf_select_blocks_1d",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
     "lf_blocks_for_sparsity", "lf_frames_selected", "lf_list_capacity", "lf_get_device_error",
     "lf_status_string", "lf_version", "HSACall",
@@ -34,6 +35,7 @@ __all__ = [
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
     "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
+    "lf_select_blocks_1d",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_block_sparse_attn_static",
     "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
 )
@@ -104,6 +106,7 @@ def _load() -> ctypes.CDLL:
         "lf_select_frames": ([S, I32, I32, P, P, P, P], I32),
         "lf_list_capacity": ([S, I32, I32, I32], I32),
         "lf_select_blocks": ([S, I32, I32, I32, P, P, P, P, P, I32, P], I32),
+        "lf_select_blocks_1d": ([S, I32, I32, P, P, P, P, I32, P], I32),
         "lf_block_sparse_attn": ([S, P, P, P, P, P, I32, F32, P, P], I32),
         "lf_block_sparse_attn_ws": ([S, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
         "lf_attn_split_plan": ([S, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
@@ -218,6 +221,17 @@ def lf_select_blocks(shape: LfShape, chunk_index: int, topk_frames: int, topk_bl
                                  _dev_ptr(block_list, torch.int32, "block_list"),
                                  _dev_ptr(block_count, torch.int32, "block_count"), list_cap,
                                  _stream(stream)), "lf_select_blocks")
+
+
+def lf_select_blocks_1d(shape: LfShape, chunk_index: int, topk_blocks: int, q_pool, k_pool,
+                        block_list, block_count, list_cap: int, stream=None) -> None:
+    import torch
+    _check(_lib.lf_select_blocks_1d(ctypes.byref(shape), chunk_index, topk_blocks,
+                                    _dev_ptr(q_pool, torch.float32, "q_pool"),
+                                    _dev_ptr(k_pool, torch.float32, "k_pool"),
+                                    _dev_ptr(block_list, torch.int32, "block_list"),
+                                    _dev_ptr(block_count, torch.int32, "block_count"), list_cap,
+                                    _stream(stream)), "lf_select_blocks_1d")
 
 
 def lf_block_sparse_attn(shape: LfShape, q, k, v, block_list, block_count, list_cap: int,

@@ -283,6 +283,28 @@ lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index, int32
     return launch_status(lf::launch_select_blocks(a, static_cast<cudaStream_t>(stream)));
 }
 
+lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_blocks,
+                              const float* q_pool, const float* k_pool, int32_t* block_list, int32_t* block_count,
+                              int32_t list_cap, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (d.Nkv > lf::SEL1D_MAX_NKV) return LF_ERR_SHAPE;
+    if (chunk_index < 1) return LF_ERR_ARG;
+    if (topk_blocks < 1) return LF_ERR_TOPK;
+    if (!q_pool || !k_pool || !block_list || !block_count) return LF_ERR_NULL;
+    if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(block_list) || !aligned16(block_count))
+        return LF_ERR_ALIGN;
+    const int keep = (chunk_index == 1 || topk_blocks > d.Nkv) ? d.Nkv : topk_blocks;
+    if (list_cap < keep) return LF_ERR_CAP;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    lf::SelectBlocks1dArgs a{q_pool, k_pool, block_list, block_count, d.B * d.H, d.D, d.Rq, d.Nkv,
+                             keep, list_cap, chunk_index};
+    return launch_status(lf::launch_select_blocks_1d(a, static_cast<cudaStream_t>(stream)));
+}
+
 lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap, int32_t sm, int32_t* tail_rows,
                              int32_t* pieces, int64_t* workspace_bytes)
 {

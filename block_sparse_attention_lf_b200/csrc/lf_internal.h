@@ -37,6 +37,18 @@ struct SelectBlocksArgs {
     int* err;
 };
 
+// One-dimensional (single-granularity) block selection: every KV block of the
+// head is a candidate; the row keeps the top `kb` of them.
+struct SelectBlocks1dArgs {
+    const float* q_pool;
+    const float* k_pool;
+    int* block_list;
+    int* block_count;
+    int BH, D, Rq, Nkv, kb, list_cap, chunk_index;
+};
+
+constexpr int SEL1D_MAX_NKV = 16384;  // candidate keys held in shared memory (128 KB)
+
 struct AttnArgs {
     const int* block_list;
     const int* block_count;
@@ -61,6 +73,7 @@ struct AttnMaps {
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s);
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s);
+cudaError_t launch_select_blocks_1d(const SelectBlocks1dArgs& a, cudaStream_t s);
 // interleaved: K/V tensor maps are the 4-D block maps (head_dim 128 only).
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s);
 

@@ -206,6 +206,94 @@ __global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const Select
     }
 }
 
+// One-dimensional selection (the single-granularity variant of the ablation in
+// "南洋理工大学打造视频生成新引擎", 163.com, section 4): one CTA per scored row,
+// every KV block of the head a candidate. Warps score groups of 32 candidates
+// into 64-bit keys in shared memory; the kb-th largest key T is built bit by
+// bit from the top (a candidate bit stays when at least kb keys are >= the
+// value with it set; keys are unique, so exactly kb keys are >= T); a ballot
+// compaction in index order writes the kept ids ascending.
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS) select_blocks_1d_kernel(const SelectBlocks1dArgs a)
+{
+    constexpr int EPL = D / 32;
+    extern __shared__ uint64_t keys[];  // [Nkv]
+    __shared__ int red[2][SEL_WARPS];   // per-warp partial counts, two alternating slots
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long row = blockIdx.x;
+    const int bh = static_cast<int>(row / a.Rq);
+    const int n = a.Nkv;
+    int* out = a.block_list + row * a.list_cap;
+    const int keep = (a.chunk_index == 1 || a.kb >= n) ? n : a.kb;
+    if (tid == 0) a.block_count[row] = keep;
+    if (keep == n) {
+        for (int g = tid; g < n; g += SEL_THREADS) out[g] = g;
+        return;
+    }
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    const float* kblk = a.k_pool + static_cast<long long>(bh) * n * D;
+    for (int grp = warp; grp * 32 < n; grp += SEL_WARPS) {
+        const float sc = score_group<D>(qv, kblk, grp * 32, n, lane);
+        const int g = grp * 32 + lane;
+        if (g < n) keys[g] = make_key(sc, g);
+    }
+    __syncthreads();
+    uint64_t T = 0;
+    for (int bit = 63; bit >= 0; --bit) {
+        const uint64_t cand = T | (1ull << bit);
+        unsigned c = 0;
+        for (int g = tid; g < n; g += SEL_THREADS) c += keys[g] >= cand ? 1u : 0u;
+        c = __reduce_add_sync(0xffffffffu, c);
+        const int buf = bit & 1;
+        if (lane == 0) red[buf][warp] = static_cast<int>(c);
+        __syncthreads();
+        int total = 0;
+#pragma unroll
+        for (int w = 0; w < SEL_WARPS; ++w) total += red[buf][w];
+        if (total >= keep) T = cand;
+    }
+    __syncthreads();  // the last round's counts are read before the slots are reused
+    int prefix = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = 0, it = 0; base < n; base += SEL_THREADS, ++it) {
+        const int g = base + tid;
+        const bool sel = g < n && keys[g] >= T;
+        const uint32_t m = __ballot_sync(0xffffffffu, sel);
+        const int buf = it & 1;
+        if (lane == 0) red[buf][warp] = __popc(m);
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < SEL_WARPS; ++w) {
+            const int v = red[buf][w];
+            total += v;
+            before += (w < warp) ? v : 0;
+        }
+        if (sel) out[prefix + before + __popc(m & lt)] = g;
+        prefix += total;
+    }
+}
+
+template <int D>
+cudaError_t launch_blocks_1d_d(const SelectBlocks1dArgs& a, cudaStream_t s)
+{
+    const size_t smem = static_cast<size_t>(a.Nkv) * sizeof(uint64_t);
+    static int configured_device = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(select_blocks_1d_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(SEL1D_MAX_NKV * sizeof(uint64_t)));
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(a.BH) * a.Rq);
+    select_blocks_1d_kernel<D><<<grid, SEL_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_frames_d(const SelectFramesArgs& a, unsigned grid, cudaStream_t s)
 {
@@ -231,6 +319,12 @@ cudaError_t launch_blocks_d(const SelectBlocksArgs& a, unsigned grid, cudaStream
 }
 
 }  // namespace
+
+cudaError_t launch_select_blocks_1d(const SelectBlocks1dArgs& a, cudaStream_t s)
+{
+    if (static_cast<long long>(a.BH) * a.Rq <= 0) return cudaSuccess;
+    return a.D == 128 ? launch_blocks_1d_d<128>(a, s) : launch_blocks_1d_d<64>(a, s);
+}
 
 cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s)
 {

@@ -14,6 +14,8 @@
  *                        plus the always-kept sink / recent / current frames
  *   lf_select_blocks     per selected frame: block scores, top-k blocks J_r(tau),
  *                        written as a compacted block list (the mask B_r)
+ *   lf_select_blocks_1d  one-dimensional variant: global block top-k over all
+ *                        KV blocks, no frame level (the ablation baseline)
  *   lf_block_sparse_attn softmax attention of each query block over the valid
  *                        tokens of its listed KV blocks (tcgen05 tensor cores)
  *   lf_block_sparse_attn_ws  the same with the last, partial wave of query
@@ -184,6 +186,27 @@ LF_API lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index
                            int32_t topk_blocks, const float* q_pool, const float* k_pool,
                            const int32_t* frame_sel, int32_t* block_list, int32_t* block_count,
                            int32_t list_cap, void* stream);
+
+/*
+ * One-dimensional (single-granularity) block selection: the variant without
+ * the frame level that the ablation of "南洋理工大学打造视频生成新引擎"
+ * (163.com, section 4) compares against. Reading (the pages name the variant
+ * without spelling it out): o_r(g) = <q~_r, k~_g> for every KV block g of the
+ * call, the row keeps the top-k of them with no frame forced in.
+ *   k_pool       [B,H,Nkv,D] fp32 from lf_pool (q_pool likewise).
+ *   topk_blocks  k >= 1; k >= Nkv, or chunk_index == 1 (dense first chunk),
+ *                keeps every block.
+ *   block_list   [B,H,Rq,list_cap] int32 out: the kept global block ids,
+ *                ascending; block_count [B,H,Rq] out: min(k, Nkv) (Nkv for
+ *                chunk 1). The lists feed lf_block_sparse_attn unchanged.
+ * Among equal scores the lower block index wins. Nkv is limited to 16384.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE (also Nkv > 16384),
+ * LF_ERR_TOPK, LF_ERR_CAP (list_cap below the kept count), LF_ERR_ARG
+ * (chunk_index < 1), LF_ERR_NO_DEVICE, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_blocks,
+                              const float* q_pool, const float* k_pool, int32_t* block_list,
+                              int32_t* block_count, int32_t list_cap, void* stream);
 
 /*
  * Block-sparse softmax attention (paper.rainbus.top, execution flow, stage 3,

@@ -117,6 +117,7 @@ def test_shape_validation(bad, code):
     assert L.lib.lf_select_frames(ctypes.byref(sh), 2, 4, p, p, p, None) == code
     assert L.lib.lf_select_blocks(ctypes.byref(sh), 2, 4, 12, p, p, p, p, p, 1000, None) == code
     assert L.lib.lf_block_sparse_attn(ctypes.byref(sh), p, p, p, p, p, 1000, 0.0, p, None) == code
+    assert L.lib.lf_select_blocks_1d(ctypes.byref(sh), 2, 12, p, p, p, p, 1000, None) == code
     assert L.lf_frames_selected(sh, 2, 4) == -1
     assert L.lf_list_capacity(sh, 2, 4, 12) == -1
 
@@ -227,3 +228,20 @@ def test_split_plan_validation():
     assert f(ctypes.byref(sh), -1, 148, ctypes.byref(t), ctypes.byref(k), ctypes.byref(b)) == 5
     assert f(ctypes.byref(sh), 108, 148, None, ctypes.byref(k), ctypes.byref(b)) == 1
     assert f(ctypes.byref(_shape(head_dim=96)), 108, 148, ctypes.byref(t), ctypes.byref(k), ctypes.byref(b)) == 3
+
+
+def test_select_1d_validation():
+    sh = _shape()  # 21 frames x 25 blocks = 525 candidates
+    p = ctypes.c_void_p(FAKE)
+    mis = ctypes.c_void_p(FAKE + 8)
+    S = ctypes.byref(sh)
+    f = L.lib.lf_select_blocks_1d
+    assert f(S, 0, 12, p, p, p, p, 108, None) == 9      # chunk index is 1-based
+    assert f(S, 2, 0, p, p, p, p, 108, None) == 4       # top-k below 1
+    assert f(S, 2, 108, None, p, p, p, 108, None) == 1
+    assert f(S, 2, 108, p, mis, p, p, 108, None) == 2
+    assert f(S, 2, 108, p, p, p, p, 107, None) == 5     # list shorter than the kept count
+    assert f(S, 1, 1, p, p, p, p, 524, None) == 5       # chunk 1 keeps all 525
+    assert f(S, 2, 10 ** 6, p, p, p, p, 524, None) == 5  # k above Nkv keeps all 525
+    big = _shape(n_frames=700, n_sink=1, n_recent=1, n_cur=3)  # 17500 candidates
+    assert f(ctypes.byref(big), 2, 12, p, p, p, p, 100, None) == 3
