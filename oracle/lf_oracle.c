@@ -35,6 +35,24 @@
  *
  * Inputs q, k, v are bf16 bit patterns (uint16). Step 1 of every routine converts
  * them to fp64 exactly; all arithmetic after that is fp64.
+ *
+ * Parity status (every routine is pinned to something other than itself by the
+ * tests named; a planted-mistake test checks that the pins catch errors):
+ *   orc_pool              pinned: hand-worked fixture, token-ramp closed form,
+ *                         constants and frame = weighted block means
+ *                         (tests/test_oracle_pool.py)
+ *   orc_frames_selected,  pinned: hand-worked fixture with ties, brute-force
+ *   orc_select_frames,    subset enumeration of top-k, invariants
+ *   orc_select_blocks     (tests/test_oracle_select.py)
+ *   orc_select_blocks_1d  pinned: brute-force top-k with ties, invariants, no
+ *                         forced frame, agreement with the two-level selection
+ *                         on frame-structured scores (tests/test_oracle_select.py)
+ *   orc_attention         pinned: all-keep mask = fp64 scaled_dot_product_attention,
+ *                         single and partial blocks, convex combination, row
+ *                         subsets, per-query-block lists (tests/test_oracle_attention.py)
+ *   orc_cag,              pinned: hand-worked budgets, the weighted-target
+ *   orc_blocks_for_sparsity  identity and growth (tests/test_oracle_cag.py)
+ * Parity with the authors' own system is unpinned: no outputs of it are given.
  */
 #include <math.h>
 #include <stdint.h>
