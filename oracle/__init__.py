@@ -49,6 +49,8 @@ def configure(lib):
     lib.orc_select_frames.restype = None
     lib.orc_select_blocks.argtypes = [_i] * 9 + [_p, _p, _p, _p, _p, _i, _p]
     lib.orc_select_blocks.restype = _i
+    lib.orc_select_frames_ivf.argtypes = [_i] * 13 + [_p, _p, _p, _p, _p]
+    lib.orc_select_frames_ivf.restype = None
     lib.orc_select_blocks_1d.argtypes = [_i] * 7 + [_p, _p, _p, _p, _i, _p]
     lib.orc_select_blocks_1d.restype = _i
     lib.orc_attention.argtypes = [_i] * 6 + [_l, _p, _p, _p, _p, _p, _i, _d, _p, _l, _p]
@@ -180,6 +182,25 @@ def select_blocks(s: Shape, chunk_index: int, topk_blocks: int, q_pool: np.ndarr
     if rc != 0:
         raise ValueError("block list exceeds list_cap")
     return lst, cnt, sc
+
+
+def select_frames_ivf(s: Shape, chunk_index: int, topk_frames: int, n_clusters: int, n_probe: int,
+                      iters: int, q_pool: np.ndarray, k_frame: np.ndarray
+                      ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Frame selection through a k-means index over the memory-frame means:
+    (T_r [B,H,Rq,n_sel] int32, centroids [B,H,C,D], labels [B,H,n_mem])."""
+    lib = _load()
+    n_sel = frames_selected(s, chunk_index, topk_frames)
+    C = max(1, min(n_clusters, s.n_mem))
+    qp = np.ascontiguousarray(q_pool, np.float64)
+    kf = np.ascontiguousarray(k_frame, np.float64)
+    sel = np.zeros((s.batch, s.heads, s.Rq, n_sel), np.int32)
+    cent = np.zeros((s.batch, s.heads, C, s.head_dim), np.float64)
+    lab = np.zeros((s.batch, s.heads, max(s.n_mem, 0)), np.int32)
+    lib.orc_select_frames_ivf(s.batch, s.heads, s.head_dim, s.Rq, s.n_frames, s.n_sink, s.n_recent,
+                              s.n_cur, chunk_index, topk_frames, n_clusters, n_probe, iters, _ptr(qp),
+                              _ptr(kf), _ptr(sel), _ptr(cent), _ptr(lab) if lab.size else None)
+    return sel, cent, lab
 
 
 def select_blocks_1d(s: Shape, chunk_index: int, topk_blocks: int, q_pool: np.ndarray,

@@ -14,6 +14,7 @@ import pytest
 import oracle
 import tests.test_oracle_attention as t_attn
 import tests.test_oracle_cag as t_cag
+import tests.test_oracle_ivf as t_ivf
 import tests.test_oracle_pool as t_pool
 import tests.test_oracle_select as t_sel
 
@@ -30,6 +31,10 @@ PINS = [
     lambda: [t_sel.test_select_1d_invariants(*a) for a in [(2, 1), (2, 7), (2, 10**6), (1, 3)]],
     t_sel.test_select_1d_forces_no_frame,
     t_sel.test_select_1d_matches_two_level_on_frame_structured_scores,
+    lambda: [t_ivf.test_ivf_full_probe_equals_exact_selection(*a) for a in [(0, 4, 3), (1, 1, 2), (2, 7, 5), (3, 10, 1)]],
+    lambda: [t_ivf.test_ivf_kmeans_matches_sklearn(s) for s in range(4)],
+    lambda: [t_ivf.test_ivf_probing_invariants(*a) for a in [(0, 5, 1, 2), (1, 5, 2, 6), (2, 8, 3, 4), (3, 3, 1, 9)]],
+    t_ivf.test_ivf_dense_first_chunk,
     lambda: [t_attn.test_all_keep_equals_dense_sdpa(*a) for a in [(100, 64, 16), (64, 64, 8)]],
     t_attn.test_single_block_and_partial_block,
     t_attn.test_rows_subset_and_empty_list,
@@ -62,6 +67,10 @@ MUTATIONS = [
     ("1-D scores the neighbouring block", "cand[g].score = dot(qr, k_pool + (bh * (long)Nkv + g) * D, D);", "cand[g].score = dot(qr, k_pool + (bh * (long)Nkv + (g + 1) % Nkv) * D, D);"),
     ("1-D list left in score order", "qsort(kept, (size_t)keep, sizeof(int), by_int);", ""),
     ("1-D first chunk not dense", "int keep = (chunk_index == 1 || topk_blocks > Nkv) ? Nkv : topk_blocks;", "int keep = topk_blocks > Nkv ? Nkv : topk_blocks;"),
+    ("IVF ranks clusters by the negated score", "cl[j].score = dot(qr, cent + (long)j * D, D);", "cl[j].score = -dot(qr, cent + (long)j * D, D);"),
+    ("IVF centroids never move", "for (int d = 0; d < D; ++d) cent[(long)j * D + d] = sum[(long)j * D + d] / (double)cnt[j];", "for (int d = 0; d < D; ++d) cent[(long)j * D + d] += 0.0 * sum[(long)j * D + d];"),
+    ("IVF distance drops the last coordinate", "                    for (int d = 0; d < D; ++d) {\n                        double t = km", "                    for (int d = 0; d + 1 < D; ++d) {\n                        double t = km"),
+    ("IVF probes one cluster too few", "if (t >= np_min && have >= kf) break;", "if (t + 1 >= np_min && have >= kf) break;"),
     ("k_b truncates instead of rounding", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel);"),
 ]
 
