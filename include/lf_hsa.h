@@ -21,6 +21,8 @@
  *   lf_block_sparse_attn_ws  the same with the last, partial wave of query
  *                        blocks split into list pieces (caller workspace)
  *   lf_attn_split_plan   that split's plan and workspace size (host only)
+ *   lf_block_sparse_attn_static  the split attention for callers that cannot
+ *                        allocate: its scratch is an array inside the library
  *
  * plus the host-side Chunk-Aware Growth budget solver (same pages, stage 1 /
  * Technical Summary 2.1).
@@ -40,7 +42,9 @@
  *   block j of KV frame tau (Nkv = n_frames*bpf blocks).
  * - bf16 data is passed as uint16_t bit patterns; pooled data is fp32.
  * - Ownership: the caller allocates every device buffer (inputs, outputs and
- *   the intermediate pooled / selection buffers). The library never allocates,
+ *   the intermediate pooled / selection buffers, the split's workspace);
+ *   lf_block_sparse_attn_static uses a fixed scratch array compiled into the
+ *   library instead. The library never allocates,
  *   frees or synchronises; each call only enqueues kernels on `stream`
  *   (a cudaStream_t; NULL = the legacy default stream) and returns.
  * - Device pointers must be 16-byte aligned (the attention kernel reads them
