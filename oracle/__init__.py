@@ -55,6 +55,16 @@ def configure(lib):
     lib.orc_select_blocks_1d.restype = _i
     lib.orc_attention.argtypes = [_i] * 6 + [_l, _p, _p, _p, _p, _p, _i, _d, _p, _l, _p]
     lib.orc_attention.restype = None
+    lib.orc_e4m3.argtypes = [_d]
+    lib.orc_e4m3.restype = _d
+    lib.orc_e4m3_array.argtypes = [_p, _l, _p]
+    lib.orc_e4m3_array.restype = None
+    lib.orc_quant_rows_e4m3.argtypes = [_p, _l, _i, _p, _p]
+    lib.orc_quant_rows_e4m3.restype = None
+    lib.orc_quant_cols_e4m3.argtypes = [_p, _l, _l, _l, _i, _p, _p]
+    lib.orc_quant_cols_e4m3.restype = None
+    lib.orc_attention_f64.argtypes = [_i] * 6 + [_l, _p, _p, _p, _p, _p, _i, _d, _p, _l, _p]
+    lib.orc_attention_f64.restype = None
     lib.orc_cag.argtypes = [_i, _p, _p, _d, _d, _i, _p, _p]
     lib.orc_cag.restype = _i
     lib.orc_blocks_for_sparsity.argtypes = [_d, _i, _i, _i]
@@ -247,6 +257,71 @@ def attention(s: Shape, q, k, v, block_list: np.ndarray, block_count: np.ndarray
     if full:
         return out.reshape(s.batch, s.heads, s.Lq, s.head_dim)
     return out
+
+
+def e4m3(x) -> np.ndarray:
+    """Nearest e4m3 value of each element (ties to even, saturating at 448), fp64."""
+    xa = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.zeros_like(xa)
+    _load().orc_e4m3_array(_ptr(xa), xa.size, _ptr(out))
+    return out
+
+
+def quant_rows_e4m3(x) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row (per token) e4m3 quantisation of bf16 x [..., D]: (dequantised fp64, scales [...])."""
+    xb = _bf16_bits(x)
+    D = xb.shape[-1]
+    n = xb.size // D
+    out = np.zeros(xb.shape, np.float64)
+    sc = np.zeros(xb.shape[:-1], np.float64)
+    _load().orc_quant_rows_e4m3(_ptr(xb), n, D, _ptr(out), _ptr(sc))
+    return out, sc
+
+
+def quant_cols_e4m3(x, rows: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-channel e4m3 quantisation of bf16 x [B,H,stride,D] over the first `rows`
+    rows of each head: (dequantised fp64 [B,H,stride,D], scales [B,H,D])."""
+    xb = _bf16_bits(x)
+    B, H, stride, D = xb.shape
+    rows = stride if rows is None else rows
+    out = np.zeros(xb.shape, np.float64)
+    sc = np.zeros((B, H, D), np.float64)
+    _load().orc_quant_cols_e4m3(_ptr(xb), B * H, rows, stride, D, _ptr(out), _ptr(sc))
+    return out, sc
+
+
+def attention_f64(s: Shape, q: np.ndarray, k: np.ndarray, v: np.ndarray, block_list: np.ndarray,
+                  block_count: np.ndarray, scale: Optional[float] = None,
+                  rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """``attention`` for fp64 inputs (q [B,H,Lq,D], k and v [B,H,kv_stride,D])."""
+    lib = _load()
+    qa, ka, va = (np.ascontiguousarray(a, np.float64) for a in (q, k, v))
+    lst = np.ascontiguousarray(block_list, np.int32)
+    cnt = np.ascontiguousarray(block_count, np.int32)
+    cap = lst.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(s.head_dim)
+    full = rows is None
+    if full:
+        rows = np.arange(s.batch * s.heads * s.Lq, dtype=np.int64)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((r.size, s.head_dim), np.float64)
+    lib.orc_attention_f64(s.batch, s.heads, s.head_dim, s.frame_tokens, s.block_tokens, s.n_cur,
+                          s.stride, _ptr(qa), _ptr(ka), _ptr(va), _ptr(lst), _ptr(cnt), cap,
+                          float(scale), _ptr(r), r.size, _ptr(out))
+    if full:
+        return out.reshape(s.batch, s.heads, s.Lq, s.head_dim)
+    return out
+
+
+def attention_fp8_inputs(s: Shape, q, k, v, block_list: np.ndarray, block_count: np.ndarray,
+                         scale: Optional[float] = None, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """``attention`` over e4m3-quantised inputs: q and k per token, v per channel of each
+    head (over the call's n_frames * frame_tokens rows); the softmax weights stay exact."""
+    qd, _ = quant_rows_e4m3(q)
+    kd, _ = quant_rows_e4m3(k)
+    vd, _ = quant_cols_e4m3(v, s.n_frames * s.frame_tokens)
+    return attention_f64(s, qd, kd, vd, block_list, block_count, scale=scale, rows=rows)
 
 
 def cag(T: Sequence[float], w: Optional[Sequence[float]], s_base: float, s_target: float,

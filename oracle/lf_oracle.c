@@ -53,6 +53,12 @@
  *   orc_attention         pinned: all-keep mask = fp64 scaled_dot_product_attention,
  *                         single and partial blocks, convex combination, row
  *                         subsets, per-query-block lists (tests/test_oracle_attention.py)
+ *   orc_e4m3,             pinned: torch's float8_e4m3fn cast on every e4m3 value,
+ *   orc_quant_rows_e4m3,  every midpoint and random values; hand-worked scaled
+ *   orc_quant_cols_e4m3   rows and columns; the largest magnitude kept exactly
+ *                         (tests/test_oracle_fp8.py)
+ *   orc_attention_f64     pinned: equal to orc_attention on bf16 inputs
+ *                         (tests/test_oracle_fp8.py)
  *   orc_cag,              pinned: hand-worked budgets, the weighted-target
  *   orc_blocks_for_sparsity  identity and growth (tests/test_oracle_cag.py)
  * Parity with the authors' own system is unpinned: no outputs of it are given.
@@ -473,6 +479,135 @@ void orc_attention(int B, int H, int D, int F, int bt, int n_cur, long kv_stride
     free(tok);
     free(z);
     free(qt);
+}
+
+/* ---- FP8 (e4m3) inputs for an FP8 attention ------------------------------ */
+/*
+ * The pages quantise linear layers to FP8 with per-channel weight scales and
+ * per-token activation scales (163.com article, deployment section; [GS]
+ * results, "FP8 linear layers"); they do not describe an FP8 attention. These
+ * routines give the inputs such an attention would see: e4m3 values times fp64
+ * scales. Readings: Q and K per token (the scale stays outside the contraction
+ * over head_dim), V per channel within a head (its contraction runs over
+ * tokens, so only a per-channel scale factors out); s = max |x| / 448 over the
+ * scaled set, 1 for an all-zero set.
+ */
+
+/* The e4m3 value nearest to x (sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, subnormals below 2^-6 in steps of 2^-9, no infinities, largest finite
+ * 448); ties go to the even mantissa; |x| beyond 448 saturates to 448. */
+double orc_e4m3(double x)
+{
+    if (x != x) return x;
+    double a = fabs(x);
+    if (a >= 448.0) return x < 0 ? -448.0 : 448.0;
+    double step;
+    if (a < ldexp(1.0, -6)) {
+        step = ldexp(1.0, -9);
+    } else {
+        int e;
+        frexp(a, &e);              /* a = f * 2^e, f in [0.5, 1): leading bit 2^(e-1) */
+        step = ldexp(1.0, e - 4);  /* 3 mantissa bits below the leading bit */
+    }
+    double qv = nearbyint(a / step) * step;  /* default rounding mode: nearest, ties to even */
+    return x < 0 ? -qv : qv;
+}
+
+/* orc_e4m3 of each of n values. */
+void orc_e4m3_array(const double* x, long n, double* out)
+{
+    for (long i = 0; i < n; ++i) out[i] = orc_e4m3(x[i]);
+}
+
+/* Row-wise (per token) e4m3 quantisation of n_rows rows of D bf16 values:
+ * out[i][d] = s_i * e4m3(x[i][d] / s_i), scales[i] = s_i (when not NULL). */
+void orc_quant_rows_e4m3(const uint16_t* x, long n_rows, int D, double* out, double* scales)
+{
+    for (long i = 0; i < n_rows; ++i) {
+        double amax = 0.0;
+        for (int d = 0; d < D; ++d) {
+            double t = fabs(bf16_to_f64(x[i * D + d]));
+            if (t > amax) amax = t;
+        }
+        double sc = amax > 0.0 ? amax / 448.0 : 1.0;
+        for (int d = 0; d < D; ++d) out[i * D + d] = sc * orc_e4m3(bf16_to_f64(x[i * D + d]) / sc);
+        if (scales) scales[i] = sc;
+    }
+}
+
+/* Column-wise (per channel) e4m3 quantisation inside each of n_groups groups
+ * (heads) of `rows` rows spaced `stride` rows apart: out has the layout of x
+ * (rows past `rows` in a group are left untouched), scales[g][d] (when not
+ * NULL). */
+void orc_quant_cols_e4m3(const uint16_t* x, long n_groups, long rows, long stride, int D, double* out,
+                         double* scales)
+{
+    for (long g = 0; g < n_groups; ++g)
+        for (int d = 0; d < D; ++d) {
+            double amax = 0.0;
+            for (long i = 0; i < rows; ++i) {
+                double t = fabs(bf16_to_f64(x[(g * stride + i) * D + d]));
+                if (t > amax) amax = t;
+            }
+            double sc = amax > 0.0 ? amax / 448.0 : 1.0;
+            for (long i = 0; i < rows; ++i)
+                out[(g * stride + i) * D + d] = sc * orc_e4m3(bf16_to_f64(x[(g * stride + i) * D + d]) / sc);
+            if (scales) scales[g * D + d] = sc;
+        }
+}
+
+/* orc_attention on fp64 inputs (q [B,H,Lq,D], k and v [B,H,kv_stride,D]): the
+ * same gather, two-pass softmax and weighted sum, for inputs that are not bf16
+ * (the dequantised FP8 values above). */
+void orc_attention_f64(int B, int H, int D, int F, int bt, int n_cur, long kv_stride,
+                       const double* q, const double* k, const double* v,
+                       const int* block_list, const int* block_count, int list_cap,
+                       double scale, const long* rows, long n_rows, double* out)
+{
+    int bpf = ceil_div(F, bt);
+    long Lq = (long)n_cur * F;
+    int Rq = n_cur * bpf;
+    (void)B; (void)H;
+    long max_tok = (long)list_cap * bt;
+    double* z = (double*)malloc(sizeof(double) * (size_t)(max_tok > 0 ? max_tok : 1));
+    long* tok = (long*)malloc(sizeof(long) * (size_t)(max_tok > 0 ? max_tok : 1));
+    for (long i = 0; i < n_rows; ++i) {
+        long bh = rows[i] / Lq;
+        long t = rows[i] % Lq;
+        int r = (int)(t / F) * bpf + (int)((t % F) / bt);
+        const double* qt = q + (bh * Lq + t) * D;
+        const int* lst = block_list + (bh * Rq + r) * (long)list_cap;
+        int cnt = block_count[bh * Rq + r];
+        long n = 0;
+        for (int c = 0; c < cnt; ++c) {
+            int g = lst[c];
+            int tau = g / bpf, j = g % bpf;
+            int t0, t1;
+            block_span(F, bt, j, &t0, &t1);
+            for (int s = t0; s < t1; ++s) tok[n++] = (long)tau * F + s;
+        }
+        double* o = out + i * (long)D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (n == 0) continue;
+        const double* kh = k + bh * kv_stride * D;
+        const double* vh = v + bh * kv_stride * D;
+        double zmax = -INFINITY;
+        for (long s = 0; s < n; ++s) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += qt[d] * kh[tok[s] * D + d];
+            z[s] = scale * acc;
+            if (z[s] > zmax) zmax = z[s];
+        }
+        double denom = 0.0;
+        for (long s = 0; s < n; ++s) {
+            double w = exp(z[s] - zmax);
+            denom += w;
+            for (int d = 0; d < D; ++d) o[d] += w * vh[tok[s] * D + d];
+        }
+        for (int d = 0; d < D; ++d) o[d] /= denom;
+    }
+    free(tok);
+    free(z);
 }
 
 /* ---- stage 1: Chunk-Aware Growth ------------------------------------------ */

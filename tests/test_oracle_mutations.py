@@ -14,6 +14,7 @@ import pytest
 import oracle
 import tests.test_oracle_attention as t_attn
 import tests.test_oracle_cag as t_cag
+import tests.test_oracle_fp8 as t_fp8
 import tests.test_oracle_ivf as t_ivf
 import tests.test_oracle_pool as t_pool
 import tests.test_oracle_select as t_sel
@@ -35,6 +36,12 @@ PINS = [
     lambda: [t_ivf.test_ivf_kmeans_matches_sklearn(s) for s in range(4)],
     lambda: [t_ivf.test_ivf_probing_invariants(*a) for a in [(0, 5, 1, 2), (1, 5, 2, 6), (2, 8, 3, 4), (3, 3, 1, 9)]],
     t_ivf.test_ivf_dense_first_chunk,
+    t_fp8.test_e4m3_matches_torch_on_values_midpoints_and_random,
+    t_fp8.test_e4m3_saturates,
+    t_fp8.test_quant_rows_hand_worked,
+    t_fp8.test_quant_cols_hand_worked_per_head,
+    lambda: [t_fp8.test_quant_keeps_the_largest_magnitude_and_the_error_bound(s) for s in range(3)],
+    t_fp8.test_attention_f64_equals_attention_on_bf16_inputs,
     lambda: [t_attn.test_all_keep_equals_dense_sdpa(*a) for a in [(100, 64, 16), (64, 64, 8)]],
     t_attn.test_single_block_and_partial_block,
     t_attn.test_rows_subset_and_empty_list,
@@ -71,6 +78,12 @@ MUTATIONS = [
     ("IVF centroids never move", "for (int d = 0; d < D; ++d) cent[(long)j * D + d] = sum[(long)j * D + d] / (double)cnt[j];", "for (int d = 0; d < D; ++d) cent[(long)j * D + d] += 0.0 * sum[(long)j * D + d];"),
     ("IVF distance drops the last coordinate", "                    for (int d = 0; d < D; ++d) {\n                        double t = km", "                    for (int d = 0; d + 1 < D; ++d) {\n                        double t = km"),
     ("IVF probes one cluster too few", "if (t >= np_min && have >= kf) break;", "if (t + 1 >= np_min && have >= kf) break;"),
+    ("e4m3 keeps four mantissa bits", "step = ldexp(1.0, e - 4);", "step = ldexp(1.0, e - 5);"),
+    ("e4m3 truncates", "double qv = nearbyint(a / step) * step;", "double qv = floor(a / step) * step;"),
+    ("e4m3 subnormal step halved", "step = ldexp(1.0, -9);", "step = ldexp(1.0, -10);"),
+    ("row scale from the first element", "double t = fabs(bf16_to_f64(x[i * D + d]));", "double t = fabs(bf16_to_f64(x[i * D]));"),
+    ("column scale from the first row", "double t = fabs(bf16_to_f64(x[(g * stride + i) * D + d]));", "double t = fabs(bf16_to_f64(x[(g * stride) * D + d]));"),
+    ("fp64 attention drops the last coordinate", "for (int d = 0; d < D; ++d) acc += qt[d] * kh[tok[s] * D + d];", "for (int d = 0; d + 1 < D; ++d) acc += qt[d] * kh[tok[s] * D + d];"),
     ("k_b truncates instead of rounding", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel);"),
 ]
 
