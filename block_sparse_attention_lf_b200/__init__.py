@@ -11,6 +11,20 @@ The library is loaded from this directory (``liblf_hsa.so``, built by
 ``build.py``); importing this module fails loudly when it is missing, and the
 device entry points raise when the tensors are not CUDA tensors. There is no
 CPU fallback.
+
+Typical use (q [B,H,n_cur*F,D], k and v [B,H,n_frames*F,D], bf16 on the GPU)::
+
+    shape = LfShape.make(B, H, D, F, n_frames, n_sink, n_recent, n_cur)
+    call = HSACall(shape, chunk_index, topk_frames, topk_blocks)
+    out = call(q, k, v)          # pool, select frames, select blocks, attend
+
+``HSACall.attend`` uses ``lf_block_sparse_attn_ws`` with a workspace sized by
+``lf_attn_split_plan`` (the split of the attention's last, partial wave);
+``tail_pieces=1`` turns the split off. ``lf_pool_range`` re-pools only some
+frames (keep the pooled keys of past frames between calls),
+``lf_select_blocks_1d`` gives the single-granularity lists of the ablation, and
+``lf_cag_budget`` / ``lf_blocks_for_sparsity`` turn a sparsity target into
+per-chunk block counts.
 """
 from __future__ import annotations
 
