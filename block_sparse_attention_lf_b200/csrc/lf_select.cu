@@ -18,6 +18,8 @@
 //   * frames: top-k by k rounds of warp arg-max over the keys;
 //   * blocks: top-k by rank counting (rank = number of larger keys), then a
 //     ballot/popc compaction writes the kept block ids in ascending order.
+// The one-dimensional variant (global block top-k, no frame level) takes one
+// CTA per scored row instead; see select_blocks_1d_kernel.
 #include "lf_device.cuh"
 #include "lf_internal.h"
 
