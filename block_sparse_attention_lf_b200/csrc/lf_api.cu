@@ -17,20 +17,18 @@ namespace {
 __device__ int g_device_error;  // first device-side fault code (0 = none)
 
 constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices] = {};
 std::mutex g_mu;
 
+// Device address of the error word on the current device. Looked up on every
+// call (a host-side table lookup once the module is loaded), so a context that
+// was torn down and re-created never leaves a stale address behind.
 lf_status error_word(int** out)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_NO_DEVICE;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_err_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return LF_ERR_CUDA;
-        g_err_ptr[dev] = static_cast<int*>(p);
-    }
-    *out = g_err_ptr[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LF_ERR_NO_DEVICE;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess || !p) return LF_ERR_CUDA;
+    *out = static_cast<int*>(p);
     return LF_OK;
 }
 
@@ -448,8 +446,12 @@ namespace {
 
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_attn_scratch on the current device (looked up once per
-// device; host code cannot use the symbol itself as a device pointer).
+// Device address of g_attn_scratch on the current device, looked up once per
+// device at the first call and kept for the life of the process (host code
+// cannot use the symbol itself as a device pointer). The kept address belongs
+// to the device's primary context: after cudaDeviceReset it is stale, so a
+// process that resets a device must not call lf_block_sparse_attn_static on it
+// again (stated in lf_hsa.h).
 lf_status static_scratch(void** out)
 {
     int dev = 0;

@@ -244,7 +244,9 @@ LF_API lf_status lf_block_sparse_attn(const lf_hsa_shape* shape, const uint16_t*
  *   tail_pieces      0: automatic plan (lf_attn_split_plan on the current
  *                    device); 1: no split; >= 2: that many pieces per list.
  *                    The piece count is lowered to what `workspace` holds and
- *                    to list_cap; below 2 nothing is split.
+ *                    to list_cap; below 2 nothing is split. (This entry point
+ *                    caps the pieces at its workspace; lf_block_sparse_attn_static,
+ *                    whose scratch is fixed, refuses a split that does not fit.)
  *   workspace        device scratch, 16-byte aligned, owned by the caller,
  *                    64 * (head_dim + 2) * 4 bytes per piece slot (r * pieces
  *                    slots); NULL with workspace_bytes == 0 means no split.
@@ -292,7 +294,9 @@ LF_API lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap,
  *                split, >= 2: that many pieces per split list).
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and keeps it; make that
- * first call before any stream capture.
+ * first call before any stream capture. The kept address belongs to the
+ * device's primary context: a process that calls cudaDeviceReset must not call
+ * this entry point on that device afterwards.
  * Sharing: every call on a device uses the same array and leaves its partial
  * rows in it. Each call writes every slot it reads before reading it, so
  * nothing has to start at zero, but two calls that overlap on the GPU (other

@@ -79,16 +79,18 @@ def _within_cut(scores: np.ndarray, chosen_idx: Sequence[int], k: int) -> bool:
 
 
 def check_frames(shape, chunk: int, kf: int, g: dict, o: dict) -> Dict[str, int]:
-    """Frame selection under the tie rule; returns counts of exact / tie rows."""
+    """Frame selection under the tie rule. Returns the number of clear rows (all equal
+    to the oracle's), of rows with an unclear cut ("tie") and of those that differ
+    from the oracle's choice ("differ", each within the cut's tolerance)."""
     gsel, osel, fsc = g["frame_sel"], o["frame_sel"], o["frame_scores"]
     assert gsel.shape == osel.shape
     if chunk == 1:
         assert (gsel == osel).all()
-        return dict(exact=gsel[..., 0].size, tie=0)
+        return dict(exact=gsel[..., 0].size, tie=0, differ=0)
     n_sink, n_mem = shape.n_sink, shape.n_mem
     forced = list(range(n_sink)) + list(range(shape.n_frames - shape.n_recent - shape.n_cur, shape.n_frames))
     k_eff = min(kf, n_mem)
-    exact = tie = 0
+    exact = tie = differ = 0
     for idx in np.ndindex(gsel.shape[:-1]):
         row_g, row_o = gsel[idx], osel[idx]
         if _clear_cut(fsc[idx], k_eff):
@@ -96,15 +98,19 @@ def check_frames(shape, chunk: int, kf: int, g: dict, o: dict) -> Dict[str, int]
             exact += 1
             continue
         tie += 1
+        if (row_g == row_o).all():
+            continue
+        differ += 1
         assert list(row_g) == sorted(set(row_g.tolist())), f"row {idx} not ascending/unique"
         assert set(forced) <= set(row_g.tolist())
         mem = [int(f) - n_sink for f in row_g if n_sink <= f < n_sink + n_mem]
         assert _within_cut(fsc[idx], mem, k_eff), f"frame tie row {idx}: {row_g}"
-    return dict(exact=exact, tie=tie)
+    return dict(exact=exact, tie=tie, differ=differ)
 
 
 def check_blocks(shape, chunk: int, kb: int, g: dict, o_q_pool, o_k_pool) -> Dict[str, int]:
-    """Block selection given the GPU's frames, under the tie rule."""
+    """Block selection given the GPU's frames, under the tie rule; returns the number of
+    rows equal to the oracle's ("exact") and of rows that differ at a tie ("tie")."""
     gsel = g["frame_sel"]
     lst_o, cnt_o, bsc = oracle.select_blocks(shape, chunk, kb, o_q_pool, o_k_pool, gsel,
                                              list_cap=g["list_cap"])

@@ -104,33 +104,63 @@ def _kb(w, shape):
     return oracle.blocks_for_sparsity(w.sparsity, shape.Nkv, n_sel, shape.bpf)
 
 
+def _head_rows(shape, bh):
+    """Every query row of (batch*head) index bh."""
+    return np.arange(bh * shape.Lq, (bh + 1) * shape.Lq, dtype=np.int64)
+
+
 @pytest.mark.parametrize("name,kb_override", [("layer480p", None), ("longvideo480p", None),
                                               ("patterns480p", None), ("patterns480p", 6)])
 def test_full_size_workloads(name, kb_override):
+    """Full size, the benchmark's launch configuration (automatic split of the last wave).
+    Every pooled value and mask row is checked; output rows: a sample of every head, the
+    split query blocks' first and last rows, and at layer480p every row of the last head
+    (4680 rows, which hold the split query blocks)."""
     w = lf_synth.CONFIGS[name]
     q, k, v = lf_synth.make_qkv(w)
     shape = oracle.shape_of(w)
     kb = kb_override or _kb(w, shape)
     rows = parity.sample_rows(shape, per_block=3, blocks_per_head=5, seed=1)
     rows = np.union1d(rows, _tail_rows(shape, w.chunk_index, w.topk_frames, kb))
+    if name == "layer480p":
+        rows = np.union1d(rows, _head_rows(shape, shape.batch * shape.heads - 1))
     fr, bl, at = _full_check(shape, q, k, v, w.chunk_index, w.topk_frames, kb, rows=rows)
-    # the planted structure makes most frame cuts clear
-    assert fr["exact"] >= 0.5 * (fr["exact"] + fr["tie"])
+    n_rows = shape.batch * shape.heads * shape.Rq
+    print(f"{name} k_b {kb}: frame rows clear {fr['exact']}, unclear {fr['tie']} "
+          f"(differing {fr['differ']}); block rows equal {bl['exact']}, differing at ties {bl['tie']}; "
+          f"max-abs {at['max_abs']:.2e} rel-Frobenius {at['rel_fro']:.2e} over {rows.size} rows")
+    # fp32 scores against fp64 ones: a choice can differ only where two candidates' scores agree
+    # to about fp32 rounding, which the planted structure makes rare; a selection fault that
+    # stays inside the tie tolerance on many rows fails here
+    assert fr["differ"] <= max(1, n_rows // 1000)
+    assert bl["tie"] <= max(1, n_rows // 1000)
 
 
 def test_rollout_chunks():
-    """The 7-chunk rollout: chunk 1 dense, chunks 2-7 with the Chunk-Aware Growth budgets."""
+    """The 7-chunk rollout: chunk 1 dense, chunks 2-7 with the Chunk-Aware Growth budgets
+    computed by the library (lf_cag_budget, lf_blocks_for_sparsity), which must equal the
+    oracle's."""
+    import block_sparse_attention_lf_b200 as L
     w = lf_synth.CONFIGS["rollout480p"]
     qa, ka, va = lf_synth.make_rollout_qkv(w)
     n_chunks = int(w.extra["n_chunks"])
+    T = list(range(1, n_chunks + 1))
+    st, s_lib, beta_lib = L.lf_cag_budget(T, T, w.extra["s_base"], w.sparsity, True)
     rc, s, beta = oracle.cag(np.arange(1, n_chunks + 1), np.arange(1, n_chunks + 1),
                              w.extra["s_base"], w.sparsity, True)
-    assert rc == 0
+    assert st == 0 and rc == 0
+    assert abs(beta_lib - beta) <= 1e-12 and np.allclose(s_lib, s, rtol=0, atol=1e-12)
     for chunk in range(1, n_chunks + 1):
         wc, q, k, v = lf_synth.rollout_chunk(w, qa, ka, va, chunk)
         shape = oracle.shape_of(wc)
-        n_sel = oracle.frames_selected(shape, chunk, w.topk_frames)
-        kb = shape.bpf if chunk == 1 else oracle.blocks_for_sparsity(s[chunk - 1], shape.Nkv, n_sel, shape.bpf)
+        ls = L.shape_from_workload(wc)
+        n_sel = L.lf_frames_selected(ls, chunk, w.topk_frames)
+        assert n_sel == oracle.frames_selected(shape, chunk, w.topk_frames)
+        if chunk == 1:
+            kb = shape.bpf
+        else:
+            kb = L.lf_blocks_for_sparsity(s_lib[chunk - 1], ls.Nkv, n_sel, ls.bpf)
+            assert kb == oracle.blocks_for_sparsity(s[chunk - 1], shape.Nkv, n_sel, shape.bpf)
         rows = parity.sample_rows(shape, per_block=2, blocks_per_head=3, seed=chunk)
         _full_check(shape, q, k, v, chunk, w.topk_frames, kb, rows=rows)
 

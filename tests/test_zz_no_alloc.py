@@ -13,7 +13,10 @@ the output tolerance of the other parity tests: two calls in a row (the second
 finds the first call's partial rows still in the array), the automatic split at
 the layer480p size, forced splits of two small cases (run after the large one,
 so the array holds another shape's rows), and the refusal of a split that needs
-more than the array holds. This file is collected last.
+more than the array holds. The layer480p output is also compared with the fp64
+oracle on sampled rows (the split rows among them), and the device's free
+memory is the same before and after a call (the entry point allocates
+nothing). This file is collected last.
 """
 import ctypes
 import os
@@ -26,6 +29,7 @@ import torch
 
 import block_sparse_attention_lf_b200 as L
 import lf_synth
+import oracle
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -66,35 +70,59 @@ def _lists(shape, chunk, kf, kb, q, k):
 
 
 def _two_calls_match(shape, q, k, v, b, tail_pieces):
+    """Two calls in a row against the existing entry point; returns the last output."""
     ref = torch.empty_like(b.out)
     assert _existing(shape, q, k, v, b, ref) == 0
     r = ref.float().cpu().numpy().astype(np.float64)
-    for _ in range(2):
-        out = torch.full_like(b.out, float("nan"))  # every row must be written
+    outs = [torch.full_like(b.out, float("nan")) for _ in range(2)]  # every row must be written
+    torch.cuda.synchronize()
+    for i, out in enumerate(outs):
+        free0 = torch.cuda.mem_get_info()[0]
         assert _static(shape, q, k, v, b, out, tail_pieces) == 0
         torch.cuda.synchronize()
+        if i == 1:
+            # the first call on the device may load the module; the next allocates nothing
+            assert torch.cuda.mem_get_info()[0] == free0, "lf_block_sparse_attn_static changed free device memory"
         st, detail = L.lf_get_device_error()
         assert st == 0, f"device error word {st} detail {detail:#x}"
         g = out.float().cpu().numpy().astype(np.float64)
         assert np.isfinite(g).all()
         assert np.abs(g - r).max() <= parity.OUT_MAX_ABS
         assert np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30) <= parity.OUT_REL_FRO
+    return outs[-1]
 
 
-def _layer480p():
+def _layer480p(host=False):
     w = lf_synth.CONFIGS["layer480p"]
     shape = L.shape_from_workload(w)
     n_sel = L.lf_frames_selected(shape, w.chunk_index, w.topk_frames)
     kb = w.topk_blocks or L.lf_blocks_for_sparsity(w.sparsity, shape.Nkv, n_sel, shape.bpf)
-    q, k, v = [t.cuda() for t in lf_synth.make_qkv(w)]
-    return shape, q, k, v, _lists(shape, w.chunk_index, w.topk_frames, kb, q, k)
+    qh, kh, vh = lf_synth.make_qkv(w)
+    q, k, v = qh.cuda(), kh.cuda(), vh.cuda()
+    b = _lists(shape, w.chunk_index, w.topk_frames, kb, q, k)
+    return (shape, q, k, v, b, (w, qh, kh, vh)) if host else (shape, q, k, v, b)
 
 
 def test_static_scratch_layer480p_two_calls():
-    shape, q, k, v, b = _layer480p()
+    shape, q, k, v, b, (w, qh, kh, vh) = _layer480p(host=True)
     tail, pieces, nbytes = L.lf_attn_split_plan(shape, b.list_cap)
     assert tail > 0 and pieces >= 2 and 0 < nbytes <= _scratch_bytes()  # the array is used
-    _two_calls_match(shape, q, k, v, b, 0)
+    out = _two_calls_match(shape, q, k, v, b, 0)
+    # the same output against the fp64 oracle on the GPU's lists: sampled rows of every head
+    # plus the first and last row of each split query block
+    s_or = oracle.shape_of(w)
+    rows = parity.sample_rows(s_or, per_block=2, blocks_per_head=3, seed=11)
+    n_rows = shape.batch * shape.heads * shape.Rq
+    split = []
+    for qb in range(n_rows - tail, n_rows):
+        bh, r = divmod(qb, shape.Rq)
+        f, j = divmod(r, shape.bpf)
+        t0 = f * shape.frame_tokens + j * 64
+        split += [bh * shape.Lq + t0, bh * shape.Lq + min(t0 + 64, (f + 1) * shape.frame_tokens) - 1]
+    rows = np.union1d(rows, np.array(split, np.int64))
+    g = dict(block_list=b.block_list.cpu().numpy(), block_count=b.block_count.cpu().numpy(),
+             out=out.float().cpu().numpy().astype(np.float64))
+    parity.check_attention(s_or, qh, kh, vh, g, rows=rows)
 
 
 @pytest.mark.parametrize("B,H,D,F,frames,chunk,kf,kb,pieces", [
