@@ -51,6 +51,10 @@ def _args():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the per-config report (all five workloads, rollout per chunk)")
     p.add_argument("--config-steps", type=int, default=30)
+    p.add_argument("--strong", action="store_true",
+                   help="N > 1: split one call's (batch, head) units across the ranks (strong scaling); "
+                        "default: each rank takes a whole workload's units of a call whose batch grows "
+                        "with N (weak scaling)")
     return p.parse_args()
 
 
@@ -165,22 +169,62 @@ def _dist():
     return None, 0, 1, 0
 
 
-def _max_over_ranks(dist, x):
+def _reduce_over_ranks(dist, x, op="max"):
     if dist is None:
         return x
     import torch
     dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
     t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
 
 
+def _max_over_ranks(dist, x):
+    return _reduce_over_ranks(dist, x, "max")
+
+
+def _idle_rank(a, dist, ws):
+    """A rank with no (batch, head) units (strong scaling with more ranks than
+    units): it takes the same collective steps as a working rank, in the same order."""
+    if dist is None:
+        return
+    dist.barrier()                       # before the timed region
+    dist.barrier()                       # after it
+    _reduce_over_ranks(dist, 0.0, "max")  # step time
+    _reduce_over_ranks(dist, 0.0, "sum")  # credited FLOPs
+    _reduce_over_ranks(dist, 0.0, "max")  # end-to-end time
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def _rank_workload(name, rank):
-    """Weak scaling: every rank runs its own independent call of the same shape
-    (different (batch, head) data: the seed is offset by the rank)."""
+    """Weak scaling: the call's batch grows with the number of ranks and rank i
+    takes the contiguous (batch, head) units [i*U, (i+1)*U), U = one workload's
+    batch*heads (shard_units of the grown call); its slice is drawn directly
+    (the workload's generator with the seed offset by the rank)."""
     import lf_synth
     w = lf_synth.CONFIGS[name]
     return w if rank == 0 else lf_synth.workload(name, seed=w.seed + 1000 * rank)
+
+
+def _rank_inputs(L, lf_synth, name, rank, ws, strong):
+    """(workload, per-rank LfShape or None, q, k, v on the host, unit range).
+    strong: one call of the workload, its (batch, head) units split across the
+    ranks (shard_shape); otherwise every rank takes a whole workload's units of a
+    call whose batch grows with the ranks."""
+    if strong and ws > 1:
+        w = lf_synth.CONFIGS[name]
+        q, k, v = lf_synth.make_qkv(w)
+        full = L.shape_from_workload(w)
+        shape, u0, u1 = L.shard_shape(full, ws, rank)
+        if shape is None:
+            return w, None, None, None, None, (u0, u1)
+        q, k, v = (L.unit_view(t, u0, u1).contiguous() for t in (q, k, v))
+        return w, shape, q, k, v, (u0, u1)
+    w = _rank_workload(name, rank)
+    U = w.batch * w.heads
+    q, k, v = lf_synth.make_qkv(w)
+    return w, L.shape_from_workload(w), q, k, v, (rank * U, (rank + 1) * U)
 
 
 def _oracle_sample(w, budget_s, q, k, v, block_list=None, block_count=None):
@@ -461,10 +505,11 @@ def run_ours(a):
     import block_sparse_attention_lf_b200 as L
     import lf_synth
 
-    w = _rank_workload(a.workload, rank)
-    shape = L.shape_from_workload(w)
+    w, shape, q_h, k_h, v_h, units = _rank_inputs(L, lf_synth, a.workload, rank, ws, a.strong)
+    if shape is None:  # more ranks than units: this rank idles but takes every collective step
+        _idle_rank(a, dist, ws)
+        return
     kb = _kb(L, shape, w)
-    q_h, k_h, v_h = lf_synth.make_qkv(w)
     q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
     call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb)
     b = call.buf
@@ -522,7 +567,8 @@ def run_ours(a):
     t_attn_warm = statistics.mean(s0.elapsed_time(s1) for s0, s1 in ew)
     t_step = mean_ms(0, 4)
     t_step_max = _max_over_ranks(dist, t_step)
-    value = ws * flops / (t_step_max * 1e-3) / 1e12
+    total_flops = _reduce_over_ranks(dist, flops, "sum")  # every rank's units
+    value = total_flops / (t_step_max * 1e-3) / 1e12
 
     # ---- end to end through the public API with pinned host buffers
     qp_, kp_, vp_ = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -552,9 +598,11 @@ def run_ours(a):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": t_step_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if (a.strong and ws > 1) else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (lf_synth, seeded; stands in for the pages' VBench 480p rollouts)",
-        "config": _config(w, kb),
+        "config": dict(_config(w, kb), global_batch=w.batch * (1 if (a.strong or ws == 1) else ws),
+                       parallelism=(f"(batch, head) units split over {ws} GPU(s), no exchange; "
+                                    f"rank 0 units [{units[0]}, {units[1]})")),
         "us_per_call": t_step_max * 1e3,
         "us_p10_p90": [_pct(step_ms, 10) * 1e3, _pct(step_ms, 90) * 1e3],
         "attn_us_warm_l2": t_attn_warm * 1e3,
@@ -571,7 +619,7 @@ def run_ours(a):
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16"],
                      "traffic": _attn_traffic(),
                      "peak_source": f"{peaks['source']} bf16 dense burst (MEASURED_PEAKS.json)"},
-        "e2e": {"value": ws * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": total_flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e},
         "gpu_launches": call.launches_per_call * a.steps,
         "clocks": clk.summary(),

@@ -43,7 +43,7 @@ __all__ = [
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
     "lf_blocks_for_sparsity", "lf_frames_selected", "lf_list_capacity", "lf_get_device_error",
     "lf_status_string", "lf_version", "HSACall",
-    "ABI_FUNCTIONS",
+    "ABI_FUNCTIONS", "shard_units", "shard_shape", "unit_view",
 ]
 
 # Names declared in include/lf_hsa.h.
@@ -392,6 +392,37 @@ class HSACall:
         self.select(stream)
         self.attend(q, k, v, stream)
         return self.buf.out
+
+
+def shard_units(batch: int, heads: int, world: int, rank: int) -> Tuple[int, int]:
+    """Contiguous range [u0, u1) of the call's batch*heads (batch, head) units that
+    process ``rank`` of ``world`` takes. Pooling, selection and attention of one unit
+    never read another unit's data, so the ranges need no exchange; their sizes
+    differ by at most one unit, and a rank past the unit count gets an empty range."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank outside the world")
+    n = batch * heads
+    return rank * n // world, (rank + 1) * n // world
+
+
+def shard_shape(shape: LfShape, world: int, rank: int) -> Tuple[Optional[LfShape], int, int]:
+    """(per-rank shape, u0, u1): the units [u0, u1) of ``shape`` as a call of their
+    own (batch 1, u1 - u0 heads, same frames and head stride); None when the range
+    is empty. The [B, H, L, D] tensors are contiguous over (batch, head), so the
+    slice is a pointer offset (``unit_view``)."""
+    u0, u1 = shard_units(shape.batch, shape.heads, world, rank)
+    if u1 == u0:
+        return None, u0, u1
+    s = LfShape.make(1, u1 - u0, shape.head_dim, shape.frame_tokens, shape.n_frames, shape.n_sink,
+                     shape.n_recent, shape.n_cur, block_tokens=shape.block_tokens, kv_stride=shape.kv_stride)
+    return s, u0, u1
+
+
+def unit_view(t, u0: int, u1: int):
+    """Units [u0, u1) of a contiguous [B, H, L, D] tensor as a [1, u1 - u0, L, D] view."""
+    if not t.is_contiguous():
+        raise ValueError("unit_view needs a contiguous tensor")
+    return t.reshape(-1, t.shape[-2], t.shape[-1])[u0:u1].unsqueeze(0)
 
 
 def shape_from_workload(w) -> LfShape:
