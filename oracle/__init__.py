@@ -61,6 +61,8 @@ def configure(lib):
     lib.orc_e4m3_array.restype = None
     lib.orc_quant_rows_e4m3.argtypes = [_p, _l, _i, _p, _p]
     lib.orc_quant_rows_e4m3.restype = None
+    lib.orc_quant_rows_e4m3_f32.argtypes = [_p, _l, _i, _p, _p]
+    lib.orc_quant_rows_e4m3_f32.restype = None
     lib.orc_quant_cols_e4m3.argtypes = [_p, _l, _l, _l, _i, _p, _p]
     lib.orc_quant_cols_e4m3.restype = None
     lib.orc_attention_f64.argtypes = [_i] * 6 + [_l, _p, _p, _p, _p, _p, _i, _d, _p, _l, _p]
@@ -276,6 +278,29 @@ def quant_rows_e4m3(x) -> Tuple[np.ndarray, np.ndarray]:
     sc = np.zeros(xb.shape[:-1], np.float64)
     _load().orc_quant_rows_e4m3(_ptr(xb), n, D, _ptr(out), _ptr(sc))
     return out, sc
+
+
+def quant_rows_e4m3_f32(x) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row e4m3 quantisation decided in fp32 (scale fl32(amax/448), code of
+    fl32(x/scale)): (dequantised fp64 [..., D], fp32 scales [...])."""
+    xb = _bf16_bits(x)
+    D = xb.shape[-1]
+    n = xb.size // D
+    out = np.zeros(xb.shape, np.float64)
+    sc = np.zeros(xb.shape[:-1], np.float32)
+    _load().orc_quant_rows_e4m3_f32(_ptr(xb), n, D, _ptr(out), _ptr(sc))
+    return out, sc
+
+
+def attention_fp8_qk(s: Shape, q, k, v, block_list: np.ndarray, block_count: np.ndarray,
+                     scale: Optional[float] = None, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """``attention`` with q and k quantised to e4m3 per token (decided in fp32, as the
+    FP8 attention kernel does) and v unchanged; the softmax weights stay exact."""
+    qd, _ = quant_rows_e4m3_f32(q)
+    kd, _ = quant_rows_e4m3_f32(k)
+    vd = _bf16_bits(v).view(np.uint16).astype(np.uint32) << 16
+    vd = vd.view(np.float32).astype(np.float64)
+    return attention_f64(s, qd, kd, vd, block_list, block_count, scale=scale, rows=rows)
 
 
 def quant_cols_e4m3(x, rows: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:

@@ -59,6 +59,11 @@
  *                         (tests/test_oracle_fp8.py)
  *   orc_attention_f64     pinned: equal to orc_attention on bf16 inputs
  *                         (tests/test_oracle_fp8.py)
+ *   orc_quant_rows_e4m3_f32  pinned: codes equal torch's float32 division and
+ *                         float8_e4m3fn cast, hand-worked rows with exact
+ *                         power-of-two scales, zero rows, agreement with the
+ *                         fp64 quantiser away from rounding midpoints
+ *                         (tests/test_oracle_fp8.py)
  *   orc_cag,              pinned: hand-worked budgets, the weighted-target
  *   orc_blocks_for_sparsity  identity and growth (tests/test_oracle_cag.py)
  * Parity with the authors' own system is unpinned: no outputs of it are given.
@@ -531,6 +536,30 @@ void orc_quant_rows_e4m3(const uint16_t* x, long n_rows, int D, double* out, dou
         }
         double sc = amax > 0.0 ? amax / 448.0 : 1.0;
         for (int d = 0; d < D; ++d) out[i * D + d] = sc * orc_e4m3(bf16_to_f64(x[i * D + d]) / sc);
+        if (scales) scales[i] = sc;
+    }
+}
+
+/* Row-wise (per token) e4m3 quantisation with the decision taken in fp32, the
+ * precision the FP8 attention kernel quantises in (where floating point decides
+ * a code, both sides decide in the same precision): per row the scale
+ * s_i = fl32(amax_i / 448) (1 for an all-zero row), each code
+ * e4m3(fl32(x / s_i)) (round to nearest even, saturating at 448), every fp32
+ * operation a single IEEE operation. out[i][d] = s_i * code (exact in fp64),
+ * scales[i] = s_i (when not NULL). */
+void orc_quant_rows_e4m3_f32(const uint16_t* x, long n_rows, int D, double* out, float* scales)
+{
+    for (long i = 0; i < n_rows; ++i) {
+        float amax = 0.0f;
+        for (int d = 0; d < D; ++d) {
+            float t = (float)fabs(bf16_to_f64(x[i * D + d]));
+            if (t > amax) amax = t;
+        }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        for (int d = 0; d < D; ++d) {
+            float y = (float)bf16_to_f64(x[i * D + d]) / sc;
+            out[i * D + d] = (double)sc * orc_e4m3((double)y);
+        }
         if (scales) scales[i] = sc;
     }
 }

@@ -114,3 +114,54 @@ def test_attention_on_fp8_inputs_stays_close():
     got = oracle.attention_fp8_inputs(s, q, k, v, lst, cnt)
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert 0.01 < rel < 0.08, rel
+
+
+# ---- quantisation decided in fp32 (the precision the FP8 attention kernel uses) -----
+
+def test_quant_rows_f32_hand_worked():
+    """amax 3.5 gives the exact scale 3.5/448 = 2^-7, so every code is e4m3(128 x):
+    0.30078125 (bf16 of 0.3) -> 38.5 -> 40 (step 4 in [32, 64)) -> 0.3125; a row whose
+    amax is 448 keeps scale 1; an all-zero row gets scale 1 and zero codes."""
+    x = torch.tensor([[3.5, -1.0, 0.3, 0.0],
+                      [448.0, -20.0, 0.0107421875, 1.0],
+                      [0.0, 0.0, 0.0, 0.0]]).to(torch.bfloat16)
+    out, sc = oracle.quant_rows_e4m3_f32(x)
+    assert sc.dtype == np.float32
+    np.testing.assert_array_equal(sc, np.array([2.0 ** -7, 1.0, 1.0], np.float32))
+    # row 1: -20 -> step 2 in [16, 32) -> -20; 0.0107421875 = 11 * 2^-10 -> subnormal step 2^-9 -> 5.5 * 2^-9
+    # ties to even -> 6 * 2^-9 = 0.01171875
+    np.testing.assert_array_equal(out, np.array([[3.5, -1.0, 0.3125, 0.0],
+                                                 [448.0, -20.0, 0.01171875, 1.0],
+                                                 [0.0, 0.0, 0.0, 0.0]]))
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_quant_rows_f32_matches_torch(seed):
+    """Against torch: fp32 amax / 448 and fp32 division (IEEE, as C float arithmetic),
+    then torch's float8_e4m3fn cast (round to nearest even) after clamping to +-448."""
+    g = torch.Generator().manual_seed(100 + seed)
+    mag = torch.exp(torch.randn(64, 1, generator=g) * 3.0)  # rows from ~1e-4 to ~1e4
+    x = (torch.randn(64, 128, generator=g) * mag).to(torch.bfloat16)
+    x[5] = 0.0
+    out, sc = oracle.quant_rows_e4m3_f32(x)
+    xf = x.float()
+    amax = xf.abs().amax(-1)
+    s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    code = (xf / s[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).float()
+    np.testing.assert_array_equal(sc, s.numpy())
+    np.testing.assert_array_equal(out, s.double().numpy()[:, None] * code.double().numpy())
+
+
+def test_quant_rows_f32_agrees_with_fp64_off_midpoints():
+    """The fp32 and fp64 decisions differ only where x / s lies within fp32 rounding of an
+    e4m3 midpoint: a handful of codes in 10^5, each one e4m3 step apart."""
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(1000, 128, generator=g).to(torch.bfloat16)
+    a, sa = oracle.quant_rows_e4m3_f32(x)
+    b, sb = oracle.quant_rows_e4m3(x)
+    np.testing.assert_allclose(sa, sb, rtol=2 ** -23)
+    ca, cb = a / sa.astype(np.float64)[:, None], b / sb[:, None]
+    differ = np.abs(ca - cb) > 1e-9
+    assert differ.sum() <= 40, differ.sum()
+    step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(cb), 2.0 ** -6))) - 3), 2.0 ** -9)
+    assert np.all(np.abs(ca - cb)[differ] <= step[differ] * (1 + 1e-12))

@@ -42,6 +42,8 @@ PINS = [
     t_fp8.test_quant_cols_hand_worked_per_head,
     lambda: [t_fp8.test_quant_keeps_the_largest_magnitude_and_the_error_bound(s) for s in range(3)],
     t_fp8.test_attention_f64_equals_attention_on_bf16_inputs,
+    t_fp8.test_quant_rows_f32_hand_worked,
+    lambda: [t_fp8.test_quant_rows_f32_matches_torch(s) for s in range(3)],
     lambda: [t_attn.test_all_keep_equals_dense_sdpa(*a) for a in [(100, 64, 16), (64, 64, 8)]],
     t_attn.test_single_block_and_partial_block,
     t_attn.test_rows_subset_and_empty_list,
@@ -85,6 +87,12 @@ MUTATIONS = [
     ("column scale from the first row", "double t = fabs(bf16_to_f64(x[(g * stride + i) * D + d]));", "double t = fabs(bf16_to_f64(x[(g * stride) * D + d]));"),
     ("fp64 attention drops the last coordinate", "for (int d = 0; d < D; ++d) acc += qt[d] * kh[tok[s] * D + d];", "for (int d = 0; d + 1 < D; ++d) acc += qt[d] * kh[tok[s] * D + d];"),
     ("k_b truncates instead of rounding", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel + 0.5);", "double x = floor((1.0 - s) * (double)n_kv_blocks / (double)n_sel);"),
+    ("fp32 quantiser scale divides by 447", "float sc = amax > 0.0f ? amax / 448.0f : 1.0f;",
+     "float sc = amax > 0.0f ? amax / 447.0f : 1.0f;"),
+    ("fp32 quantiser multiplies by the scale", "float y = (float)bf16_to_f64(x[i * D + d]) / sc;",
+     "float y = (float)bf16_to_f64(x[i * D + d]) * sc;"),
+    ("fp32 quantiser amax of signed values", "float t = (float)fabs(bf16_to_f64(x[i * D + d]));",
+     "float t = (float)bf16_to_f64(x[i * D + d]);"),
 ]
 
 
