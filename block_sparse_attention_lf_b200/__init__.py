@@ -39,7 +39,7 @@ LIB_PATH = os.path.join(_HERE, "liblf_hsa.so")
 
 __all__ = [
     "LfShape", "LfError", "lib", "lf_pool", "lf_pool_range", "lf_select_frames", "lf_select_blocks",
-    "lf_select_blocks_1d",
+    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf", "FrameIndex",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
     "lf_blocks_for_sparsity", "lf_frames_selected", "lf_list_capacity", "lf_get_device_error",
     "lf_status_string", "lf_version", "HSACall",
@@ -49,7 +49,7 @@ __all__ = [
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
     "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
-    "lf_select_blocks_1d",
+    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_block_sparse_attn_static",
     "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
 )
@@ -121,6 +121,8 @@ def _load() -> ctypes.CDLL:
         "lf_list_capacity": ([S, I32, I32, I32], I32),
         "lf_select_blocks": ([S, I32, I32, I32, P, P, P, P, P, I32, P], I32),
         "lf_select_blocks_1d": ([S, I32, I32, P, P, P, P, I32, P], I32),
+        "lf_frame_index_build": ([S, I32, I32, P, P, P, P, P, P], I32),
+        "lf_select_frames_ivf": ([S, I32, I32, I32, I32, P, P, P, P, P, P, P], I32),
         "lf_block_sparse_attn": ([S, P, P, P, P, P, I32, F32, P, P], I32),
         "lf_block_sparse_attn_ws": ([S, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
         "lf_attn_split_plan": ([S, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32),
@@ -246,6 +248,55 @@ def lf_select_blocks_1d(shape: LfShape, chunk_index: int, topk_blocks: int, q_po
                                     _dev_ptr(block_list, torch.int32, "block_list"),
                                     _dev_ptr(block_count, torch.int32, "block_count"), list_cap,
                                     _stream(stream)), "lf_select_blocks_1d")
+
+
+@dataclass
+class FrameIndex:
+    """Device buffers of a coarse frame index (lf_frame_index_build): fp32 centroids
+    [B,H,n_clusters,D], int32 labels and members [B,H,max(n_mem,1)], int32 offsets
+    [B,H,n_clusters+1]."""
+    n_clusters: int
+    centroids: "object"
+    labels: "object"
+    offsets: "object"
+    members: "object"
+
+    @classmethod
+    def empty(cls, shape: LfShape, n_clusters: int, device="cuda") -> "FrameIndex":
+        import torch
+        n_mem = max(shape.n_frames - shape.n_sink - shape.n_recent - shape.n_cur, 1)
+        bh = (shape.batch, shape.heads)
+        return cls(n_clusters,
+                   torch.empty(*bh, n_clusters, shape.head_dim, dtype=torch.float32, device=device),
+                   torch.empty(*bh, n_mem, dtype=torch.int32, device=device),
+                   torch.empty(*bh, n_clusters + 1, dtype=torch.int32, device=device),
+                   torch.empty(*bh, n_mem, dtype=torch.int32, device=device))
+
+
+def lf_frame_index_build(shape: LfShape, k_frame, index: FrameIndex, iters: int = 25, stream=None) -> None:
+    """k-means index over each head's memory-frame means (k_frame from lf_pool)."""
+    import torch
+    i32 = torch.int32
+    _check(_lib.lf_frame_index_build(ctypes.byref(shape), int(index.n_clusters), int(iters),
+                                     _dev_ptr(k_frame, torch.float32, "k_frame"),
+                                     _dev_ptr(index.centroids, torch.float32, "centroids"),
+                                     _dev_ptr(index.labels, i32, "labels"), _dev_ptr(index.offsets, i32, "offsets"),
+                                     _dev_ptr(index.members, i32, "members"), _stream(stream)),
+           "lf_frame_index_build")
+
+
+def lf_select_frames_ivf(shape: LfShape, chunk_index: int, topk_frames: int, index: FrameIndex, n_probe: int,
+                         q_pool, k_frame, frame_sel, stream=None) -> None:
+    """Frame selection probing the index (same output layout as lf_select_frames)."""
+    import torch
+    i32 = torch.int32
+    _check(_lib.lf_select_frames_ivf(ctypes.byref(shape), chunk_index, topk_frames, int(index.n_clusters),
+                                     int(n_probe), _dev_ptr(q_pool, torch.float32, "q_pool"),
+                                     _dev_ptr(k_frame, torch.float32, "k_frame"),
+                                     _dev_ptr(index.centroids, torch.float32, "centroids"),
+                                     _dev_ptr(index.offsets, i32, "offsets"), _dev_ptr(index.members, i32, "members"),
+                                     _dev_ptr(frame_sel, i32, "frame_sel"), _stream(stream)),
+           "lf_select_frames_ivf")
 
 
 def lf_block_sparse_attn(shape: LfShape, q, k, v, block_list, block_count, list_cap: int,

@@ -303,6 +303,43 @@ lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, in
     return launch_status(lf::launch_select_blocks_1d(a, static_cast<cudaStream_t>(stream)));
 }
 
+lf_status lf_frame_index_build(const lf_hsa_shape* shape, int32_t n_clusters, int32_t iters, const float* k_frame,
+                               float* centroids, int32_t* labels, int32_t* offsets, int32_t* members, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (n_clusters < 1 || n_clusters > lf::IVF_MAX_CLUSTERS || iters < 0 || iters > 100000) return LF_ERR_ARG;
+    if (!k_frame || !centroids || !labels || !offsets || !members) return LF_ERR_NULL;
+    if (!aligned16(k_frame) || !aligned16(centroids) || !aligned16(labels) || !aligned16(offsets) ||
+        !aligned16(members))
+        return LF_ERR_ALIGN;
+    const int C = std::min(n_clusters, std::max(d.n_mem, 1));
+    lf::FrameIndexArgs a{k_frame, centroids, labels, offsets, members, d.B * d.H, d.D, d.NF, d.n_sink, d.n_mem,
+                         C, n_clusters, std::max(d.n_mem, 1), iters};
+    return launch_status(lf::launch_frame_index(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_select_frames_ivf(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, int32_t n_clusters,
+                               int32_t n_probe, const float* q_pool, const float* k_frame, const float* centroids,
+                               const int32_t* offsets, const int32_t* members, int32_t* frame_sel, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (chunk_index < 1 || n_clusters < 1 || n_clusters > lf::IVF_MAX_CLUSTERS || n_probe < 1) return LF_ERR_ARG;
+    if (topk_frames < 1) return LF_ERR_TOPK;
+    if (!q_pool || !k_frame || !centroids || !offsets || !members || !frame_sel) return LF_ERR_NULL;
+    if (!aligned16(q_pool) || !aligned16(k_frame) || !aligned16(centroids) || !aligned16(offsets) ||
+        !aligned16(members) || !aligned16(frame_sel))
+        return LF_ERR_ALIGN;
+    const int C = std::min(n_clusters, std::max(d.n_mem, 1));
+    lf::SelectFramesIvfArgs a{q_pool, k_frame, centroids, offsets, members, frame_sel, d.B * d.H, d.D, d.Rq, d.NF,
+                              d.n_sink, d.n_recent, d.n_cur, d.n_mem, frames_selected(d, chunk_index, topk_frames),
+                              topk_frames, chunk_index, C, n_clusters, std::max(d.n_mem, 1), std::min(n_probe, C)};
+    return launch_status(lf::launch_select_frames_ivf(a, static_cast<cudaStream_t>(stream)));
+}
+
 lf_status lf_attn_split_plan(const lf_hsa_shape* shape, int32_t list_cap, int32_t sm, int32_t* tail_rows,
                              int32_t* pieces, int64_t* workspace_bytes)
 {

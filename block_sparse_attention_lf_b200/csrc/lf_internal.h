@@ -49,6 +49,31 @@ struct SelectBlocks1dArgs {
 
 constexpr int SEL1D_MAX_NKV = 16384;  // candidate keys held in shared memory (128 KB)
 
+// Coarse frame retrieval: a k-means index over each head's memory-frame means.
+constexpr int IVF_MAX_CLUSTERS = 64;
+constexpr int IVF_MAX_MEM = 1024;  // memory frames per call (the shape limit)
+
+struct FrameIndexArgs {
+    const float* k_frame;  // [BH, NF, D]
+    float* centroids;      // [BH, C_stride, D]: rows [0, C) written
+    int* labels;           // [BH, m_stride]: cluster of each memory frame
+    int* offsets;          // [BH, C_stride + 1]: members of cluster j are members[offsets[j], offsets[j+1])
+    int* members;          // [BH, m_stride]: memory-frame indices grouped by cluster, ascending in a cluster
+    int BH, D, NF, n_sink, n_mem, C, C_stride, m_stride, iters;
+};
+
+struct SelectFramesIvfArgs {
+    const float* q_pool;
+    const float* k_frame;
+    const float* centroids;
+    const int* offsets;
+    const int* members;
+    int* frame_sel;
+    int BH, D, Rq, NF, n_sink, n_recent, n_cur, n_mem, n_sel, topk, chunk_index, C, C_stride, m_stride, n_probe;
+};
+
+size_t frame_index_smem_bytes(int C, int n_mem, int D);
+
 struct AttnArgs {
     const int* block_list;
     const int* block_count;
@@ -74,6 +99,8 @@ cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s);
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s);
 cudaError_t launch_select_blocks_1d(const SelectBlocks1dArgs& a, cudaStream_t s);
+cudaError_t launch_frame_index(const FrameIndexArgs& a, cudaStream_t s);
+cudaError_t launch_select_frames_ivf(const SelectFramesIvfArgs& a, cudaStream_t s);
 // interleaved: K/V tensor maps are the 4-D block maps (head_dim 128 only).
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s);
 

@@ -1,0 +1,338 @@
+// lf_ivf.cu -- coarse frame retrieval for very long videos ("Light Forcing：通过稀疏注意力
+// 加速自回归视频扩散", paper.rainbus.top, weaknesses paragraph, point 2: the frame
+// candidate set grows linearly with the video, and a hierarchical index is the remedy
+// it names; the selection it approximates is the first level of stage 3 of the
+// execution flow, p_r = <q~_r, k^_M> and top-k frames T_r).
+//
+// The pages do not fix the index. Reading taken here (the same as the oracle's):
+//   * build, once per head and whenever frames are appended: k-means with squared L2
+//     distance over the head's memory-frame means k^_m, C = min(n_clusters, |M|)
+//     clusters started at memory frames floor(i*|M|/C); Lloyd rounds until no
+//     assignment changes, at most `iters` updates (then a last assignment); an empty
+//     cluster keeps its centroid; ties go to the lower cluster;
+//   * selection, per query block: clusters ordered by <q~_r, c_j> (ties to the lower
+//     cluster); the best n_probe are probed, and further clusters in that order until
+//     the probed ones hold min(k_f, |M|) frames; the exact top-k_f of the probed
+//     clusters' frames (ties to the lower frame), plus the sink, recent and
+//     current-chunk frames, ascending. Probing every cluster is the exact selection.
+//
+// Build: one CTA per (batch, head). The k-means runs in fp64 on the fp32 frame means
+// with the oracle's operation order (distances summed over head_dim in order, member
+// sums in frame order, IEEE divisions, no fused multiply-adds), so given the same frame
+// means its labels and centroids are the oracle's, bit for bit. The result is written
+// as fp32 centroids, labels and a CSR member list grouped by cluster.
+// Selection: one warp per query block, like the exact frame selection: the centroid
+// and frame scores are fp32 inner products formed exactly as there, so with every
+// cluster probed the two kernels choose the same frames.
+#include "lf_device.cuh"
+#include "lf_internal.h"
+#include "lf_score.cuh"
+
+namespace lf {
+namespace {
+
+constexpr int IDX_THREADS = 256;
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
+
+// ---- index build ---------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(IDX_THREADS) frame_index_kernel(const FrameIndexArgs a)
+{
+    extern __shared__ double dsm[];
+    double* cent = dsm;                          // [C][D]
+    double* sum = cent + a.C * D;                // [C][D]
+    int* lab = reinterpret_cast<int*>(sum + a.C * D);  // [n_mem]
+    int* cnt = lab + a.n_mem;                    // [C]
+    int* off = cnt + a.C;                        // [C + 1]
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.x;
+    const int n = a.n_mem, C = a.C;
+    const float* km = a.k_frame + (static_cast<long long>(bh) * a.NF + a.n_sink) * D;
+
+    for (int i = tid; i < C * D; i += IDX_THREADS) {
+        const int j = i / D, d = i - j * D;
+        cent[i] = static_cast<double>(km[static_cast<long long>(j) * n / C * D + d]);
+    }
+    for (int m = tid; m < n; m += IDX_THREADS) lab[m] = -1;
+    __syncthreads();
+    for (int it = 0; it <= a.iters; ++it) {
+        int changed = 0;
+        for (int m = tid; m < n; m += IDX_THREADS) {
+            const float* x = km + static_cast<long long>(m) * D;
+            int best = 0;
+            double bd = 0.0;
+            for (int j = 0; j < C; ++j) {
+                const double* c = cent + j * D;
+                double d2 = 0.0;
+#pragma unroll 8
+                for (int d = 0; d < D; ++d) {
+                    const double t = __dsub_rn(static_cast<double>(x[d]), c[d]);
+                    d2 = __dadd_rn(d2, __dmul_rn(t, t));
+                }
+                if (j == 0 || d2 < bd) {
+                    bd = d2;
+                    best = j;
+                }
+            }
+            if (lab[m] != best) {
+                lab[m] = best;
+                changed = 1;
+            }
+        }
+        if (!__syncthreads_or(changed) || it == a.iters) break;  // converged, or the last assignment
+        // member sums in frame order: thread d owns column d of every cluster
+        for (int i = tid; i < C * D; i += IDX_THREADS) sum[i] = 0.0;
+        if (tid < C) cnt[tid] = 0;
+        __syncthreads();
+        if (tid < D) {
+            for (int m = 0; m < n; ++m) {
+                const int j = lab[m];
+                sum[j * D + tid] = __dadd_rn(sum[j * D + tid], static_cast<double>(km[static_cast<long long>(m) * D + tid]));
+            }
+        }
+        if (tid == IDX_THREADS - 1) {  // outside the column loop (D <= 128 < IDX_THREADS)
+            for (int m = 0; m < n; ++m) cnt[lab[m]] += 1;
+        }
+        __syncthreads();
+        for (int i = tid; i < C * D; i += IDX_THREADS) {
+            const int j = i / D;
+            if (cnt[j] > 0) cent[i] = __ddiv_rn(sum[i], static_cast<double>(cnt[j]));
+        }
+        __syncthreads();
+    }
+    // outputs: fp32 centroids, labels, and the members grouped by cluster (ascending inside)
+    float* co = a.centroids + static_cast<long long>(bh) * a.C_stride * D;
+    for (int i = tid; i < C * D; i += IDX_THREADS) co[i] = static_cast<float>(cent[i]);
+    int* lo = a.labels + static_cast<long long>(bh) * a.m_stride;
+    for (int m = tid; m < n; m += IDX_THREADS) lo[m] = lab[m];
+    if (tid < C) cnt[tid] = 0;
+    __syncthreads();
+    if (tid == 0) {
+        for (int m = 0; m < n; ++m) cnt[lab[m]] += 1;
+        off[0] = 0;
+        for (int j = 0; j < C; ++j) off[j + 1] = off[j] + cnt[j];
+    }
+    __syncthreads();
+    int* oo = a.offsets + static_cast<long long>(bh) * (a.C_stride + 1);
+    for (int j = tid; j <= C; j += IDX_THREADS) oo[j] = off[j];
+    // warp w compacts clusters w, w + 8, ...: ballot over the frames in order
+    int* mo = a.members + static_cast<long long>(bh) * a.m_stride;
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int j = warp; j < C; j += IDX_THREADS / 32) {
+        int pos = off[j];
+        for (int base = 0; base < n; base += 32) {
+            const int m = base + lane;
+            const bool in = m < n && lab[m] == j;
+            const uint32_t mask = __ballot_sync(0xffffffffu, in);
+            if (in) mo[pos + __popc(mask & lt)] = m;
+            pos += __popc(mask);
+        }
+    }
+}
+
+// ---- probed selection ---------------------------------------------------------
+// Scores of 32 candidate rows: candidate c is row `row_of_c` (held by lane c; < 0 = none)
+// of `rows` (D floats each); returns the score of the lane's own candidate. The partial
+// products and the reduction tree are the exact frame selection's, so a frame scores the
+// same bits in both kernels.
+template <int D>
+__device__ __forceinline__ float score_rows(const float (&qv)[D / 32], const float* rows, int row_of_lane, int lane)
+{
+    constexpr int EPL = D / 32;
+    float part[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        part[c] = 0.f;
+        const int rc = __shfl_sync(0xffffffffu, row_of_lane, c);
+        if (rc >= 0) {
+            float kv[EPL];
+            load_lane<EPL>(kv, rows + static_cast<long long>(rc) * D + lane * EPL);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) part[c] = fmaf(qv[e], kv[e], part[c]);
+        }
+    }
+    transpose_reduce_sum(part, lane);
+    return part[0];
+}
+
+__device__ __forceinline__ int* a_cand_smem()
+{
+    extern __shared__ int cand_smem[];
+    return cand_smem;
+}
+
+// KPL = candidate key slots per lane (ceil(n_mem / 32)); clusters <= 64 (two slots).
+// Dynamic shared memory: a candidate list of IVF_MAX_MEM frame indices per warp.
+template <int D, int KPL>
+__global__ void __launch_bounds__(SEL_THREADS) select_frames_ivf_kernel(const SelectFramesIvfArgs a)
+{
+    constexpr int EPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
+    if (row >= static_cast<long long>(a.BH) * a.Rq) return;
+    int* out = a.frame_sel + row * a.n_sel;
+    if (a.chunk_index == 1) {
+        for (int t = lane; t < a.NF; t += 32) out[t] = t;
+        return;
+    }
+    const int bh = static_cast<int>(row / a.Rq);
+    const int n_mem = a.n_mem, C = a.C;
+    const int kf = a.topk < n_mem ? a.topk : n_mem;
+    for (int t = lane; t < a.n_sink; t += 32) out[t] = t;
+    const int tail0 = a.NF - a.n_recent - a.n_cur;
+    for (int t = lane; t < a.n_recent + a.n_cur; t += 32) out[a.n_sink + kf + t] = tail0 + t;
+    if (n_mem == 0) return;
+
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    const float* cent = a.centroids + static_cast<long long>(bh) * a.C_stride * D;
+    const int* off = a.offsets + static_cast<long long>(bh) * (a.C_stride + 1);
+    const int* mem = a.members + static_cast<long long>(bh) * a.m_stride;
+    const float* kmem = a.k_frame + (static_cast<long long>(bh) * a.NF + a.n_sink) * D;
+
+    // 1. clusters in score order; probe at least n_probe and until kf frames are held
+    uint64_t ck[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int j = 32 * i + lane;
+        const float sc = score_rows<D>(qv, cent, j < C ? j : -1, lane);
+        ck[i] = j < C ? make_key(sc, j) : 0ull;
+    }
+    uint64_t probed = 0;  // bit j: cluster j is probed (same in every lane)
+    int have = 0;
+    for (int t = 0; t < C; ++t) {
+        if (t >= a.n_probe && have >= kf) break;
+        const uint64_t best = warp_max_u64(ck[0] > ck[1] ? ck[0] : ck[1]);
+        const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+        probed |= 1ull << j;
+        have += max(0, min(__ldg(off + j + 1), n_mem) - max(__ldg(off + j), 0));
+        if (ck[0] == best) ck[0] = 0ull;
+        if (ck[1] == best) ck[1] = 0ull;
+    }
+
+    // 2. the probed clusters' frames, gathered into this warp's candidate list
+    int* cand = a_cand_smem() + (threadIdx.x >> 5) * IVF_MAX_MEM;
+    int nc = 0;
+    for (uint64_t pb = probed; pb; pb &= pb - 1) {
+        const int j = __ffsll(static_cast<long long>(pb)) - 1;
+        // an index built for this shape has 0 <= offsets[j] <= offsets[j+1] <= n_mem; other
+        // values are clamped so a wrong buffer cannot send a read out of bounds
+        const int b = min(max(__ldg(off + j), 0), n_mem);
+        const int e = min(max(__ldg(off + j + 1), b), n_mem);
+        const int take = min(e - b, IVF_MAX_MEM - nc);
+        for (int p = lane; p < take; p += 32) {
+            const int m = __ldg(mem + b + p);
+            cand[nc + p] = (m >= 0 && m < n_mem) ? m : -1;
+        }
+        nc += take;
+    }
+    __syncwarp();
+    // candidate 32 g + l is key slot g of lane l; keys carry the frame index, so they are unique
+    uint64_t key[KPL];
+#pragma unroll
+    for (int g = 0; g < KPL; ++g) {
+        key[g] = 0ull;
+        if (32 * g < nc) {
+            const int m = 32 * g + lane < nc ? cand[32 * g + lane] : -1;  // -1: no candidate
+            const float sc = score_rows<D>(qv, kmem, m, lane);
+            if (m >= 0) key[g] = make_key(sc, m);
+        }
+    }
+
+    // 3. top-kf by warp arg-max rounds; chosen frame m is bit m / 32 of lane m % 32
+    uint32_t sel = 0;
+    for (int t = 0; t < kf; ++t) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int g = 0; g < KPL; ++g) best = key[g] > best ? key[g] : best;
+        const uint64_t wbest = warp_max_u64(best);
+        if (wbest == 0ull) break;
+#pragma unroll
+        for (int g = 0; g < KPL; ++g)
+            if (key[g] == wbest) key[g] = 0ull;
+        const int m = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(wbest));
+        if ((m & 31) == lane) sel |= 1u << (m >> 5);
+    }
+    int prefix = a.n_sink;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const bool s = (sel >> i) & 1u;
+        const uint32_t mask = __ballot_sync(0xffffffffu, s);
+        if (s) out[prefix + __popc(mask & lt)] = a.n_sink + i * 32 + lane;
+        prefix += __popc(mask);
+    }
+}
+
+template <int D, int KPL>
+cudaError_t launch_ivf_select_k(const SelectFramesIvfArgs& a, unsigned grid, cudaStream_t s)
+{
+    constexpr size_t smem = static_cast<size_t>(SEL_WARPS) * IVF_MAX_MEM * sizeof(int);
+    static int configured_device = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(select_frames_ivf_kernel<D, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    select_frames_ivf_kernel<D, KPL><<<grid, SEL_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_ivf_select_d(const SelectFramesIvfArgs& a, unsigned grid, cudaStream_t s)
+{
+    const int kpl = (a.n_mem + 31) / 32;
+    if (a.chunk_index == 1 || kpl <= 1) return launch_ivf_select_k<D, 1>(a, grid, s);
+    if (kpl <= 2) return launch_ivf_select_k<D, 2>(a, grid, s);
+    if (kpl <= 4) return launch_ivf_select_k<D, 4>(a, grid, s);
+    if (kpl <= 8) return launch_ivf_select_k<D, 8>(a, grid, s);
+    if (kpl <= 16) return launch_ivf_select_k<D, 16>(a, grid, s);
+    return launch_ivf_select_k<D, 32>(a, grid, s);
+}
+
+template <int D>
+cudaError_t launch_index_d(const FrameIndexArgs& a, cudaStream_t s)
+{
+    const size_t smem = frame_index_smem_bytes(a.C, a.n_mem, D);
+    static int configured_device = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(frame_index_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(frame_index_smem_bytes(IVF_MAX_CLUSTERS, IVF_MAX_MEM, D)));
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    frame_index_kernel<D><<<static_cast<unsigned>(a.BH), IDX_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t frame_index_smem_bytes(int C, int n_mem, int D)
+{
+    return static_cast<size_t>(2) * C * D * sizeof(double) + static_cast<size_t>(n_mem + 2 * C + 1) * sizeof(int);
+}
+
+cudaError_t launch_frame_index(const FrameIndexArgs& a, cudaStream_t s)
+{
+    if (a.BH <= 0 || a.n_mem <= 0) return cudaSuccess;
+    return a.D == 128 ? launch_index_d<128>(a, s) : launch_index_d<64>(a, s);
+}
+
+cudaError_t launch_select_frames_ivf(const SelectFramesIvfArgs& a, cudaStream_t s)
+{
+    const long long rows = static_cast<long long>(a.BH) * a.Rq;
+    if (rows <= 0) return cudaSuccess;
+    const unsigned grid = static_cast<unsigned>((rows + SEL_WARPS - 1) / SEL_WARPS);
+    return a.D == 128 ? launch_ivf_select_d<128>(a, grid, s) : launch_ivf_select_d<64>(a, grid, s);
+}
+
+}  // namespace lf

@@ -4,14 +4,16 @@
 // Technical Summary 2.2 "Token Compression").
 //
 // HBM-bound. One CTA per (batch*head, frame): the pooled K frames first, then
-// the query frames of the current chunk. Warp w of the CTA owns blocks w, w+8, w+16, ...
-// of its frame and streams each block (64 tokens x head_dim bf16, 16 KB,
-// contiguous) with 128-bit coalesced loads, 16 per lane in flight; a block's
-// column sums are reduced with warp shuffles only, so no CTA-wide barrier sits
-// between loads and 64 KB per CTA stay in flight. The frame sum is each warp's
-// running sum of its block sums, combined across the 8 warps in a fixed order
-// through shared memory once at the end (deterministic), then divided by the
-// frame's token count, so K is read once.
+// the query frames of the current chunk. The CTA has W warps, W chosen so that it
+// divides the frame's block count where possible (5 for the 25 blocks of a 1560-token
+// frame), so every warp streams the same number of blocks and none idles at the end.
+// Warp w owns blocks w, w+W, w+2W, ... and streams each block (64 tokens x head_dim
+// bf16, 16 KB, contiguous) with 128-bit coalesced loads, 16 per lane in flight; a
+// block's column sums are reduced with warp shuffles only, so no CTA-wide barrier
+// sits between loads. Several small CTAs share an SM, which keeps about 100 KB per SM
+// in flight. The frame sum is each warp's running sum of its block sums, combined
+// across the warps in a fixed order through shared memory once at the end
+// (deterministic), then divided by the frame's token count, so K is read once.
 #include "lf_internal.h"
 
 #include <cuda_bf16.h>
@@ -19,8 +21,7 @@
 namespace lf {
 namespace {
 
-constexpr int POOL_THREADS = 256;
-constexpr int POOL_WARPS = POOL_THREADS / 32;
+constexpr int POOL_MAX_WARPS = 8;
 constexpr int BLOCK_TOKENS = 64;
 
 __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p)
@@ -43,7 +44,7 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& u)
 }
 
 template <int D>
-__global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
+__global__ void __launch_bounds__(POOL_MAX_WARPS * 32) pool_kernel(const PoolArgs a)
 {
     constexpr int CPR = D / 8;          // 16-byte chunks per token row
     constexpr int RPL = 32 / CPR;       // rows one warp-wide load covers
@@ -51,7 +52,8 @@ __global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
     constexpr int PHASE = 16;           // loads in flight per lane
     static_assert(LOADS % PHASE == 0, "layout");
 
-    __shared__ float red[POOL_WARPS][D];
+    __shared__ float red[POOL_MAX_WARPS][D];
+    const int n_warps = blockDim.x >> 5;
 
     const int units = a.nk + (a.pool_q ? a.n_cur : 0);
     const int bh = blockIdx.x / units;
@@ -73,7 +75,7 @@ __global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
     const int chunk = lane % CPR, rsub = lane / CPR;
     float facc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // this warp's share of the frame sum
 
-    for (int j = warp; j < a.bpf; j += POOL_WARPS) {
+    for (int j = warp; j < a.bpf; j += n_warps) {
         const int nrows = min(BLOCK_TOKENS, a.F - j * BLOCK_TOKENS);
         const uint16_t* bsrc = src + static_cast<long long>(j) * BLOCK_TOKENS * D + chunk * 8;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -107,24 +109,41 @@ __global__ void __launch_bounds__(POOL_THREADS, 2) pool_kernel(const PoolArgs a)
         for (int i = 0; i < 8; ++i) red[warp][chunk * 8 + i] = facc[i];
     }
     __syncthreads();
-    if (threadIdx.x < D) {
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
         float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < POOL_WARPS; ++w) s += red[w][threadIdx.x];
-        a.k_frame[(static_cast<long long>(bh) * a.NF + f) * D + threadIdx.x] = s / static_cast<float>(a.F);
+        for (int w = 0; w < n_warps; ++w) s += red[w][c];
+        a.k_frame[(static_cast<long long>(bh) * a.NF + f) * D + c] = s / static_cast<float>(a.F);
     }
 }
 
 }  // namespace
 
+// Warps per CTA: the count in 4..8 that leaves the fewest idle warp-blocks over the
+// frame's bpf blocks (ties to more warps); frames of fewer than 4 blocks get one warp
+// per block. bpf = 25 gives 5 (no idle warp), bpf = 24 gives 8, bpf = 4 gives 4.
+int pool_warps(int bpf)
+{
+    if (bpf < 4) return bpf < 1 ? 1 : bpf;
+    int best = POOL_MAX_WARPS, waste = 1 << 30;
+    for (int w = POOL_MAX_WARPS; w >= 4; --w) {
+        const int idle = ((bpf + w - 1) / w) * w - bpf;
+        if (idle < waste) {
+            waste = idle;
+            best = w;
+        }
+    }
+    return best;
+}
+
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s)
 {
     const long long grid = static_cast<long long>(a.BH) * (a.nk + (a.pool_q ? a.n_cur : 0));
     if (grid <= 0) return cudaSuccess;
+    const int threads = 32 * pool_warps(a.bpf);
     if (a.D == 128)
-        pool_kernel<128><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
+        pool_kernel<128><<<static_cast<unsigned>(grid), threads, 0, s>>>(a);
     else
-        pool_kernel<64><<<static_cast<unsigned>(grid), POOL_THREADS, 0, s>>>(a);
+        pool_kernel<64><<<static_cast<unsigned>(grid), threads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -16,6 +16,9 @@
  *                        written as a compacted block list (the mask B_r)
  *   lf_select_blocks_1d  one-dimensional variant: global block top-k over all
  *                        KV blocks, no frame level (the ablation baseline)
+ *   lf_frame_index_build / lf_select_frames_ivf  coarse frame retrieval: a
+ *                        k-means index over the frame means, probed per query
+ *                        block (for very long videos)
  *   lf_block_sparse_attn softmax attention of each query block over the valid
  *                        tokens of its listed KV blocks (tcgen05 tensor cores)
  *   lf_block_sparse_attn_ws  the same with the last, partial wave of query
@@ -211,6 +214,51 @@ LF_API lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index
 LF_API lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_blocks,
                               const float* q_pool, const float* k_pool, int32_t* block_list,
                               int32_t* block_count, int32_t list_cap, void* stream);
+
+/*
+ * Coarse frame retrieval for very long videos: an index over the frame means.
+ * "Light Forcing：通过稀疏注意力加速自回归视频扩散" (paper.rainbus.top,
+ * weaknesses paragraph, point 2) notes that the frame candidates grow linearly
+ * with the video and names a hierarchical index as the remedy without fixing
+ * it. Reading taken: per (batch, head), k-means with squared L2 distance over
+ * the memory-frame means k^_m (the slice [n_sink, n_sink + n_mem) of k_frame),
+ * C = min(n_clusters, n_mem) clusters started at memory frames floor(i*n_mem/C),
+ * Lloyd rounds until no assignment changes or `iters` updates were made (then
+ * one last assignment); an empty cluster keeps its centroid; equal distances go
+ * to the lower cluster. Computed in fp64 from the fp32 frame means. Build it
+ * once per head and again when frames are appended (it does not depend on q).
+ *   n_clusters  1..64; iters 0..100000.
+ *   centroids   [B,H,n_clusters,D] fp32 out (rows [0, C) written)
+ *   labels      [B,H,max(n_mem,1)] int32 out: the cluster of each memory frame
+ *   offsets     [B,H,n_clusters+1] int32 out: cluster j holds
+ *               members[offsets[j] .. offsets[j+1])
+ *   members     [B,H,max(n_mem,1)] int32 out: memory-frame indices (0-based in
+ *               M) grouped by cluster, ascending within a cluster
+ * One CTA per (batch, head). All pointers 16-byte aligned.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_ARG, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_frame_index_build(const lf_hsa_shape* shape, int32_t n_clusters, int32_t iters,
+                               const float* k_frame, float* centroids, int32_t* labels,
+                               int32_t* offsets, int32_t* members, void* stream);
+
+/*
+ * Frame-level selection through the index of lf_frame_index_build (same
+ * passages). Per query block: clusters ordered by <q~_r, c_j> (equal scores:
+ * lower cluster first); the best n_probe are probed, and further ones in that
+ * order until the probed clusters hold min(topk_frames, n_mem) frames; T_r is
+ * the exact top-k of the probed clusters' frames by p_r = <q~_r, k^_m> (equal
+ * scores: lower frame) plus the sink, recent and current-chunk frames,
+ * ascending, in the layout of lf_select_frames (lf_select_blocks consumes it
+ * unchanged). With every cluster probed the result is lf_select_frames' result
+ * (same fp32 scores). chunk_index == 1 selects every frame.
+ *   n_clusters  the value given to lf_frame_index_build; n_probe >= 1.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE, LF_ERR_TOPK, LF_ERR_ARG,
+ * LF_ERR_CUDA.
+ */
+LF_API lf_status lf_select_frames_ivf(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames,
+                               int32_t n_clusters, int32_t n_probe, const float* q_pool,
+                               const float* k_frame, const float* centroids, const int32_t* offsets,
+                               const int32_t* members, int32_t* frame_sel, void* stream);
 
 /*
  * Block-sparse softmax attention (paper.rainbus.top, execution flow, stage 3,

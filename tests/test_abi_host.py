@@ -245,3 +245,25 @@ def test_select_1d_validation():
     assert f(S, 2, 10 ** 6, p, p, p, p, 524, None) == 5  # k above Nkv keeps all 525
     big = _shape(n_frames=700, n_sink=1, n_recent=1, n_cur=3)  # 17500 candidates
     assert f(ctypes.byref(big), 2, 12, p, p, p, p, 100, None) == 3
+
+
+def test_frame_index_validation():
+    """lf_frame_index_build / lf_select_frames_ivf reject bad arguments before launching."""
+    import ctypes
+    s = L.LfShape.make(1, 2, 128, 1560, 21, 1, 1, 3)
+    P = ctypes.c_void_p
+    p16 = P(4096)
+    ok_ptrs = [p16] * 5
+    # n_clusters outside 1..64, negative iters
+    assert L.lib.lf_frame_index_build(ctypes.byref(s), 0, 5, *ok_ptrs, None) == 9
+    assert L.lib.lf_frame_index_build(ctypes.byref(s), 65, 5, *ok_ptrs, None) == 9
+    assert L.lib.lf_frame_index_build(ctypes.byref(s), 8, -1, *ok_ptrs, None) == 9
+    assert L.lib.lf_frame_index_build(ctypes.byref(s), 8, 5, p16, None, p16, p16, p16, None) == 1
+    assert L.lib.lf_frame_index_build(ctypes.byref(s), 8, 5, P(4100), p16, p16, p16, p16, None) == 2
+    bad = L.LfShape.make(1, 2, 96, 1560, 21, 1, 1, 3)
+    assert L.lib.lf_frame_index_build(ctypes.byref(bad), 8, 5, *ok_ptrs, None) == 3
+    sel_ptrs = [p16] * 6
+    assert L.lib.lf_select_frames_ivf(ctypes.byref(s), 2, 4, 8, 0, *sel_ptrs, None) == 9   # n_probe < 1
+    assert L.lib.lf_select_frames_ivf(ctypes.byref(s), 0, 4, 8, 2, *sel_ptrs, None) == 9   # chunk < 1
+    assert L.lib.lf_select_frames_ivf(ctypes.byref(s), 2, 0, 8, 2, *sel_ptrs, None) == 4   # top-k < 1
+    assert L.lib.lf_select_frames_ivf(ctypes.byref(s), 2, 4, 8, 2, p16, p16, p16, p16, p16, None, None) == 1
