@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """Benchmark of one Light Forcing HSA attention call on B200.
 
-A step is one whole HSA call on resident inputs: block/frame mean pooling,
-frame selection, block selection and block-sparse attention (four kernels of
-liblf_hsa.so, called through the C ABI, plus the merge kernel when the
-attention splits the lists of its last, partial wave). The default workload is the
+A step is one whole HSA call on resident inputs: block/frame mean pooling, the
+two-level selection (frames, then blocks, in one launch) and block-sparse
+attention (three kernels of liblf_hsa.so, called through the C ABI, plus the
+merge kernel when the attention splits the lists of the tail). The default workload is the
 480p-shaped layer call (batch 1, 12 heads, head_dim 128, 1560-token frames,
 21 KV frames = sink + 16 memory + recent + 3-frame current chunk, frame top-4,
 block top-k for 80 % block sparsity), drawn by ``lf_synth``.
@@ -363,10 +363,8 @@ def measure_call(L, shape, chunk_index, topk_frames, kb, q, k, v, steps, warmup,
         e[0].record(stream)
         pool()
         e[1].record(stream)
-        L.lf_select_frames(shape, chunk_index, topk_frames, b.q_pool, b.k_frame, b.frame_sel)
+        call.select()
         e[2].record(stream)
-        L.lf_select_blocks(shape, chunk_index, topk_frames, kb, b.q_pool, b.k_pool, b.frame_sel,
-                           b.block_list, b.block_count, b.list_cap)
         e[3].record(stream)
         call.attend(q, k, v)
         e[4].record(stream)
@@ -383,7 +381,7 @@ def measure_call(L, shape, chunk_index, topk_frames, kb, q, k, v, steps, warmup,
     if cached:
         kf = k.numel() * nc // nf
         pool_bytes = (q.numel() + kf) * 2 + (b.q_pool.numel() + (b.k_pool.numel() + b.k_frame.numel()) * nc // nf) * 4
-    return dict(pool=us(0, 1), select_frames=us(1, 2), select_blocks=us(2, 3), attn=us(3, 4),
+    return dict(pool=us(0, 1), select=us(1, 2), attn=us(3, 4),
                 total=us(0, 4), flops=flops, pool_bytes=pool_bytes, kb=kb,
                 list_entries=int(b.block_count.sum().item()))
 
@@ -393,13 +391,13 @@ def _summary(m, peaks):
     att = m["attn"][0]
     return {
         "us_per_call": round(t, 2), "us_p10_p90": [round(m["total"][1], 2), round(m["total"][2], 2)],
-        "kernels_us": {k: round(m[k][0], 2) for k in ("pool", "select_frames", "select_blocks", "attn")},
+        "kernels_us": {k: round(m[k][0], 2) for k in ("pool", "select", "attn")},
         "kept_tflop": round(m["flops"] / 1e12, 5), "topk_blocks": m["kb"],
         "tflops_call": round(m["flops"] / (t * 1e-6) / 1e12, 1),
         "attn_tflops": round(m["flops"] / (att * 1e-6) / 1e12, 1),
         "attn_frac_of_bf16_peak": round(m["flops"] / (att * 1e-6) / 1e12 / peaks["bf16"], 4),
         "pool_frac_of_hbm": round(m["pool_bytes"] / (m["pool"][0] * 1e-6) / 1e9 / peaks["hbm"], 3),
-        "select_over_attn": round((m["pool"][0] + m["select_frames"][0] + m["select_blocks"][0]) / att, 4),
+        "select_over_attn": round((m["pool"][0] + m["select"][0]) / att, 4),
     }
 
 
@@ -537,10 +535,8 @@ def run_ours(a):
             e[0].record(stream)
             call.pool(q, k)
             e[1].record(stream)
-            L.lf_select_frames(shape, w.chunk_index, w.topk_frames, b.q_pool, b.k_frame, b.frame_sel)
+            call.select()
             e[2].record(stream)
-            L.lf_select_blocks(shape, w.chunk_index, w.topk_frames, kb, b.q_pool, b.k_pool,
-                               b.frame_sel, b.block_list, b.block_count, b.list_cap)
             e[3].record(stream)
             call.attend(q, k, v)
             e[4].record(stream)
@@ -555,7 +551,7 @@ def run_ours(a):
     def mean_ms(i0, i1):
         return statistics.mean(E[s][i0].elapsed_time(E[s][i1]) for s in range(a.steps))
 
-    t_pool, t_sf, t_sb, t_attn = mean_ms(0, 1), mean_ms(1, 2), mean_ms(2, 3), mean_ms(3, 4)
+    t_pool, t_sel, t_attn = mean_ms(0, 1), mean_ms(1, 2), mean_ms(3, 4)
     step_ms = [E[s][0].elapsed_time(E[s][4]) for s in range(a.steps)]
     # attention alone, back to back with a warm L2 (K/V of the call stay resident)
     ew = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
@@ -606,15 +602,14 @@ def run_ours(a):
         "us_per_call": t_step_max * 1e3,
         "us_p10_p90": [_pct(step_ms, 10) * 1e3, _pct(step_ms, 90) * 1e3],
         "attn_us_warm_l2": t_attn_warm * 1e3,
-        "kernels_us": {"pool": t_pool * 1e3, "select_frames": t_sf * 1e3,
-                       "select_blocks": t_sb * 1e3, "block_sparse_attn": t_attn * 1e3},
+        "kernels_us": {"pool": t_pool * 1e3, "select": t_sel * 1e3, "block_sparse_attn": t_attn * 1e3},
         "kept_tflop_per_call": flops / 1e12,
         "attn_tflops": attn_tflops,
         "attn_frac_of_bf16_peak": attn_tflops / peaks["bf16"],
         "pool_gbs": pool_bytes / (t_pool * 1e-3) / 1e9,
         "pool_frac_of_hbm": pool_bytes / (t_pool * 1e-3) / 1e9 / peaks["hbm"],
-        "select_gbs": sel_bytes / ((t_sf + t_sb) * 1e-3) / 1e9,
-        "select_over_attn": (t_pool + t_sf + t_sb) / t_attn,
+        "select_gbs": sel_bytes / (t_sel * 1e-3) / 1e9,
+        "select_over_attn": (t_pool + t_sel) / t_attn,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16"],
                      "traffic": _attn_traffic(),

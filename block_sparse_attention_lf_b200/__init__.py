@@ -39,7 +39,8 @@ LIB_PATH = os.path.join(_HERE, "liblf_hsa.so")
 
 __all__ = [
     "LfShape", "LfError", "lib", "lf_pool", "lf_pool_range", "lf_select_frames", "lf_select_blocks",
-    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf", "FrameIndex",
+    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf", "FrameIndex", "lf_select_mask",
+    "lf_quant_fp8_rows", "lf_block_sparse_attn_fp8",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_cag_budget",
     "lf_blocks_for_sparsity", "lf_frames_selected", "lf_list_capacity", "lf_get_device_error",
     "lf_status_string", "lf_version", "HSACall",
@@ -49,7 +50,8 @@ __all__ = [
 # Names declared in include/lf_hsa.h.
 ABI_FUNCTIONS = (
     "lf_pool", "lf_pool_range", "lf_frames_selected", "lf_select_frames", "lf_list_capacity", "lf_select_blocks",
-    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf",
+    "lf_select_blocks_1d", "lf_frame_index_build", "lf_select_frames_ivf", "lf_select_mask", "lf_quant_fp8_rows",
+    "lf_block_sparse_attn_fp8",
     "lf_block_sparse_attn", "lf_block_sparse_attn_ws", "lf_attn_split_plan", "lf_block_sparse_attn_static",
     "lf_cag_budget", "lf_blocks_for_sparsity", "lf_get_device_error", "lf_status_string", "lf_version",
 )
@@ -122,6 +124,9 @@ def _load() -> ctypes.CDLL:
         "lf_select_blocks": ([S, I32, I32, I32, P, P, P, P, P, I32, P], I32),
         "lf_select_blocks_1d": ([S, I32, I32, P, P, P, P, I32, P], I32),
         "lf_frame_index_build": ([S, I32, I32, P, P, P, P, P, P], I32),
+        "lf_select_mask": ([S, I32, I32, I32, P, P, P, P, P, P, I32, P], I32),
+        "lf_quant_fp8_rows": ([P, ctypes.c_int64, I32, P, P, P], I32),
+        "lf_block_sparse_attn_fp8": ([S, P, P, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
         "lf_select_frames_ivf": ([S, I32, I32, I32, I32, P, P, P, P, P, P, P], I32),
         "lf_block_sparse_attn": ([S, P, P, P, P, P, I32, F32, P, P], I32),
         "lf_block_sparse_attn_ws": ([S, P, P, P, P, P, I32, F32, P, I32, P, ctypes.c_int64, P], I32),
@@ -239,6 +244,27 @@ def lf_select_blocks(shape: LfShape, chunk_index: int, topk_frames: int, topk_bl
                                  _stream(stream)), "lf_select_blocks")
 
 
+def lf_select_mask(shape: LfShape, chunk_index: int, topk_frames: int, topk_blocks: int, q_pool, k_frame, k_pool,
+                   frame_sel, block_list, block_count, list_cap: int, stream=None) -> None:
+    """Both selection levels in one launch (the results of lf_select_frames + lf_select_blocks)."""
+    import torch
+    f32, i32 = torch.float32, torch.int32
+    _check(_lib.lf_select_mask(ctypes.byref(shape), chunk_index, topk_frames, topk_blocks,
+                               _dev_ptr(q_pool, f32, "q_pool"), _dev_ptr(k_frame, f32, "k_frame"),
+                               _dev_ptr(k_pool, f32, "k_pool"), _dev_ptr(frame_sel, i32, "frame_sel"),
+                               _dev_ptr(block_list, i32, "block_list"), _dev_ptr(block_count, i32, "block_count"),
+                               list_cap, _stream(stream)), "lf_select_mask")
+
+
+def lf_quant_fp8_rows(x, x8, scales, stream=None) -> None:
+    """Per-row e4m3 codes (uint8 tensor shaped like x) and fp32 scales (x.shape[:-1]) of bf16 x."""
+    import torch
+    D = x.shape[-1]
+    n = x.numel() // D
+    _check(_lib.lf_quant_fp8_rows(_dev_ptr(x, _bf16(), "x"), n, D, _dev_ptr(x8, torch.uint8, "x8"),
+                                  _dev_ptr(scales, torch.float32, "scales"), _stream(stream)), "lf_quant_fp8_rows")
+
+
 def lf_select_blocks_1d(shape: LfShape, chunk_index: int, topk_blocks: int, q_pool, k_pool,
                         block_list, block_count, list_cap: int, stream=None) -> None:
     import torch
@@ -328,6 +354,22 @@ def lf_block_sparse_attn_ws(shape: LfShape, q, k, v, block_list, block_count, li
            "lf_block_sparse_attn_ws")
 
 
+def lf_block_sparse_attn_fp8(shape: LfShape, q8, k8, q_scale, k_scale, v, block_list, block_count, list_cap: int,
+                             softmax_scale: float, out, workspace=None, tail_pieces: int = 0, stream=None) -> None:
+    """Attention with e4m3 q8 / k8 (uint8 codes from lf_quant_fp8_rows) and fp32 per-token scales."""
+    import torch
+    bf = _bf16()
+    u8, f32, i32 = torch.uint8, torch.float32, torch.int32
+    ws = _dev_ptr(workspace, u8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(_lib.lf_block_sparse_attn_fp8(ctypes.byref(shape), _dev_ptr(q8, u8, "q8"), _dev_ptr(k8, u8, "k8"),
+                                         _dev_ptr(q_scale, f32, "q_scale"), _dev_ptr(k_scale, f32, "k_scale"),
+                                         _dev_ptr(v, bf, "v"), _dev_ptr(block_list, i32, "block_list"),
+                                         _dev_ptr(block_count, i32, "block_count"), list_cap, float(softmax_scale),
+                                         _dev_ptr(out, bf, "out"), int(tail_pieces), ws, ws_bytes, _stream(stream)),
+           "lf_block_sparse_attn_fp8")
+
+
 def lf_attn_split_plan(shape: LfShape, list_cap: int, sm: int = 0) -> Tuple[int, int, int]:
     """(tail query blocks, pieces per list, workspace bytes) of the automatic split."""
     t, p, b = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int64(0)
@@ -371,7 +413,8 @@ class HSABuffers:
 
 
 class HSACall:
-    """One HSA call's device buffers plus the four device steps, in order.
+    """One HSA call's device buffers plus the device steps, in order: pooling, the
+    two-level selection (one launch, lf_select_mask) and the attention.
 
     ``shape``: an ``LfShape``; ``chunk_index`` is 1-based (chunk 1 is dense);
     ``topk_frames`` / ``topk_blocks`` as in the C ABI. ``tail_pieces`` selects
@@ -419,8 +462,8 @@ class HSACall:
         ws_bytes = tail * pieces * 64 * (D + 2) * 4
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes else None
         self.split = (tail, pieces) if ws_bytes else (0, 0)
-        # kernels enqueued per call: pool, two selections, attention (+ the merge of a split)
-        self.launches_per_call = 4 + (1 if ws_bytes else 0)
+        # kernels enqueued per call: pool, selection (both levels), attention (+ the merge of a split)
+        self.launches_per_call = 3 + (1 if ws_bytes else 0)
 
     def pool(self, q, k, stream=None):
         b = self.buf
@@ -428,10 +471,8 @@ class HSACall:
 
     def select(self, stream=None):
         b = self.buf
-        lf_select_frames(self.shape, self.chunk_index, self.topk_frames, b.q_pool, b.k_frame,
-                         b.frame_sel, stream)
-        lf_select_blocks(self.shape, self.chunk_index, self.topk_frames, self.topk_blocks, b.q_pool,
-                         b.k_pool, b.frame_sel, b.block_list, b.block_count, b.list_cap, stream)
+        lf_select_mask(self.shape, self.chunk_index, self.topk_frames, self.topk_blocks, b.q_pool, b.k_frame,
+                       b.k_pool, b.frame_sel, b.block_list, b.block_count, b.list_cap, stream)
 
     def attend(self, q, k, v, stream=None):
         b = self.buf

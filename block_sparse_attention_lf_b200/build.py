@@ -7,7 +7,7 @@ import sys
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_HERE)
-SOURCES = ["lf_api.cu", "lf_pool.cu", "lf_select.cu", "lf_ivf.cu", "lf_attn.cu"]
+SOURCES = ["lf_api.cu", "lf_pool.cu", "lf_select.cu", "lf_ivf.cu", "lf_quant.cu", "lf_attn.cu"]
 HEADERS = ["lf_device.cuh", "lf_internal.h", "lf_score.cuh"]
 LIB = os.path.join(_HERE, "liblf_hsa.so")
 

@@ -163,6 +163,22 @@ bool encode_rows(CUtensorMap* m, const void* base, long long rows, int D, int bo
     return r == CUDA_SUCCESS;
 }
 
+// 2-D uint8 view [rows, 128] (e4m3 rows of head_dim 128) with a {128, box_rows} box and
+// 128-byte swizzle: one box is a block of e4m3 rows.
+bool encode_rows_u8(CUtensorMap* m, const void* base, long long rows, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {128u, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {128u};
+    const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 4-D bf16 view of a [rows, 128] tensor as {64 elems, 8 rows, 2 panels,
 // rows/8 groups} with a {64, 8, 2, groups} box: one box brings a block of
 // 8*groups rows in the interleaved [group][panel][8 rows x 128 B] layout.
@@ -230,8 +246,10 @@ lf_status lf_pool_range(const lf_hsa_shape* shape, const uint16_t* q, const uint
     if (!k || !k_pool || !k_frame || (pool_q && (!q || !q_pool))) return LF_ERR_NULL;
     if (!aligned16(k) || !aligned16(k_pool) || !aligned16(k_frame) || (pool_q && (!aligned16(q) || !aligned16(q_pool))))
         return LF_ERR_ALIGN;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
     lf::PoolArgs a{q, k, q_pool, k_pool, k_frame, d.B * d.H, d.D, d.F, d.bpf, d.NF, d.n_cur, d.kv_stride,
-                   frame_begin, frame_end - frame_begin, pool_q ? 1 : 0};
+                   frame_begin, frame_end - frame_begin, pool_q ? 1 : 0, err};
     return launch_status(lf::launch_pool(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -279,6 +297,42 @@ lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index, int32
     lf::SelectBlocksArgs a{q_pool, k_pool, frame_sel, block_list, block_count, d.B * d.H, d.D, d.Rq, d.NF,
                            d.bpf, n_sel, kb, list_cap, chunk_index, err};
     return launch_status(lf::launch_select_blocks(a, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_select_mask(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames, int32_t topk_blocks,
+                         const float* q_pool, const float* k_frame, const float* k_pool, int32_t* frame_sel,
+                         int32_t* block_list, int32_t* block_count, int32_t list_cap, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (chunk_index < 1) return LF_ERR_ARG;
+    if (topk_frames < 1 || topk_blocks < 1) return LF_ERR_TOPK;
+    if (!q_pool || !k_frame || !k_pool || !frame_sel || !block_list || !block_count) return LF_ERR_NULL;
+    if (!aligned16(q_pool) || !aligned16(k_frame) || !aligned16(k_pool) || !aligned16(frame_sel) ||
+        !aligned16(block_list) || !aligned16(block_count))
+        return LF_ERR_ALIGN;
+    const int n_sel = frames_selected(d, chunk_index, topk_frames);
+    const int kb = blocks_per_frame(d, chunk_index, topk_blocks);
+    if (list_cap < n_sel * kb) return LF_ERR_CAP;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
+    lf::SelectFramesArgs fa{q_pool, k_frame, frame_sel, d.B * d.H, d.D, d.Rq, d.NF, d.n_sink, d.n_recent,
+                            d.n_cur, n_sel, topk_frames, chunk_index};
+    lf::SelectBlocksArgs ba{q_pool, k_pool, frame_sel, block_list, block_count, d.B * d.H, d.D, d.Rq, d.NF,
+                            d.bpf, n_sel, kb, list_cap, chunk_index, err};
+    return launch_status(lf::launch_select_fused(fa, ba, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_quant_fp8_rows(const uint16_t* x, int64_t n_rows, int32_t head_dim, uint8_t* x8, float* scales,
+                            void* stream)
+{
+    if (n_rows < 0 || (head_dim != 64 && head_dim != 128)) return LF_ERR_ARG;
+    if (n_rows == 0) return LF_OK;
+    if (!x || !x8 || !scales) return LF_ERR_NULL;
+    if (!aligned16(x) || !aligned16(x8) || !aligned16(scales)) return LF_ERR_ALIGN;
+    if (n_rows >= (1ll << 31) * 8) return LF_ERR_SHAPE;
+    return launch_status(lf::launch_quant_rows(x, n_rows, head_dim, x8, scales, static_cast<cudaStream_t>(stream)));
 }
 
 lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_blocks,
@@ -412,9 +466,63 @@ lf_status lf_block_sparse_attn_ws(const lf_hsa_shape* shape, const uint16_t* q, 
     float* part_o = static_cast<float*>(workspace);
     float* part_ml = pieces ? part_o + static_cast<long long>(tail) * pieces * 64 * d.D : nullptr;
     lf::AttnArgs a{block_list, block_count, out, list_cap, d.Rq, d.bpf, d.F, d.Lq, d.Nkv, d.rem, d.kv_stride,
-                   scale * 1.4426950408889634f, err, static_cast<int>(n_rows - tail), pieces, part_o, part_ml};
-    return launch_status(
-        lf::launch_attn(m, a, d.D, interleaved, static_cast<int>(n_rows), static_cast<cudaStream_t>(stream)));
+                   scale * 1.4426950408889634f, err, static_cast<int>(n_rows - tail), pieces, part_o, part_ml,
+                   static_cast<int>(n_rows), static_cast<int>(n_rows - tail + static_cast<long long>(tail) * pieces)};
+    return launch_status(lf::launch_attn(m, a, d.D, interleaved, static_cast<cudaStream_t>(stream)));
+}
+
+lf_status lf_block_sparse_attn_fp8(const lf_hsa_shape* shape, const uint8_t* q8, const uint8_t* k8,
+                                   const float* q_scale, const float* k_scale, const uint16_t* v,
+                                   const int32_t* block_list, const int32_t* block_count, int32_t list_cap,
+                                   float softmax_scale, uint16_t* out, int32_t tail_pieces, void* workspace,
+                                   int64_t workspace_bytes, void* stream)
+{
+    Derived d;
+    lf_status st = check_shape(shape, &d);
+    if (st != LF_OK) return st;
+    if (d.D != 128) return LF_ERR_SHAPE;
+    if (list_cap < 0) return LF_ERR_CAP;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return LF_ERR_ARG;
+    if (tail_pieces < 0 || workspace_bytes < 0) return LF_ERR_ARG;
+    if (!q8 || !k8 || !q_scale || !k_scale || !v || !block_list || !block_count || !out) return LF_ERR_NULL;
+    if (workspace_bytes > 0 && !workspace) return LF_ERR_NULL;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v) ||
+        !aligned16(block_list) || !aligned16(block_count) || !aligned16(out) ||
+        (workspace_bytes > 0 && !aligned16(workspace)))
+        return LF_ERR_ALIGN;
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LF_ERR_NO_DEVICE;
+    if (major != 10 || minor != 0) return LF_ERR_NO_DEVICE;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d.D));
+    const long long BH = static_cast<long long>(d.B) * d.H;
+    lf::AttnMaps m;
+    const long long q_rows = BH * d.Lq, kv_rows = BH * d.kv_stride;
+    if (!encode_rows_u8(&m.q, q8, q_rows, 64) || !encode_rows_u8(&m.q_rem, q8, q_rows, d.rem) ||
+        !encode_rows_u8(&m.k, k8, kv_rows, 64) || !encode_rows_u8(&m.k_rem, k8, kv_rows, d.rem))
+        return LF_ERR_CUDA;
+    const bool v_il = d.F % 8 == 0 && d.kv_stride % 8 == 0 && encode_blocks_il(&m.v, v, kv_rows, 8) &&
+                      encode_blocks_il(&m.v_rem, v, kv_rows, d.rem / 8);
+    if (!v_il && (!encode_rows(&m.v, v, kv_rows, d.D, 64) || !encode_rows(&m.v_rem, v, kv_rows, d.D, d.rem)))
+        return LF_ERR_CUDA;
+    const long long n_rows = BH * d.Rq;
+    int tail = 0, pieces = 0;
+    if (workspace_bytes > 0 && tail_pieces != 1) {
+        int sm = 0;
+        if ((st = sm_count(&sm)) != LF_OK) return st;
+        split_plan(n_rows, sm, list_cap, tail_pieces, workspace_bytes / split_slot_bytes(d.D), &tail, &pieces);
+    }
+    float* part_o = static_cast<float*>(workspace);
+    float* part_ml = pieces ? part_o + static_cast<long long>(tail) * pieces * 64 * d.D : nullptr;
+    lf::AttnArgs a{block_list, block_count, out, list_cap, d.Rq, d.bpf, d.F, d.Lq, d.Nkv, d.rem, d.kv_stride,
+                   scale * 1.4426950408889634f, err, static_cast<int>(n_rows - tail), pieces, part_o, part_ml,
+                   static_cast<int>(n_rows), static_cast<int>(n_rows - tail + static_cast<long long>(tail) * pieces),
+                   q_scale, k_scale};
+    return launch_status(lf::launch_attn_fp8(m, a, v_il, static_cast<cudaStream_t>(stream)));
 }
 
 lf_status lf_cag_budget(int32_t n_chunks, const double* T, const double* flops_w, double s_base, double s_target,

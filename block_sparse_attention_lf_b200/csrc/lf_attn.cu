@@ -72,8 +72,10 @@ namespace {
 
 constexpr int ATTN_THREADS = 384;
 constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_PV = 3, W_SOFT0 = 4;
-constexpr int KSLOTS = 2;   // K ring: tiles of two blocks
-constexpr int VSLOTS = 4;   // V ring: single blocks
+// K ring (tiles of two blocks) and V ring (single blocks). e4m3 K tiles take half the
+// bytes of bf16 ones, which leaves room for a deeper V ring.
+template <bool F8> struct Rings { static constexpr int K = 2, V = 4; };
+template <> struct Rings<true> { static constexpr int K = 2, V = 6; };
 constexpr int SBUFS = 3;    // S buffers in TMEM (one per step in flight)
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
 constexpr uint32_t TMEM_COLS = 512;         // S buffer b: columns 128*b; O^T of warpgroup g: 384 + 64*g
@@ -82,13 +84,16 @@ constexpr int LIST_SMEM = 1024;             // list entries staged in shared mem
 
 // Shared-memory plan. IL selects the interleaved K/V layout (head_dim 128,
 // one 4-D box per block); otherwise K/V use [panel][rows x 128 B].
-template <int D, bool IL>
+template <int D, bool IL, bool F8 = false>
 struct AttnLayout {
-    static constexpr int NP = D / 64;                    // 64-element panels of head_dim
+    static constexpr int KSLOTS = Rings<F8>::K;
+    static constexpr int VSLOTS = Rings<F8>::V;
+    static constexpr int NP = D / 64;                    // 64-element panels of head_dim (bf16)
+    static constexpr int NPQ = F8 ? 1 : NP;               // 128-byte panels of a Q / K row
     static constexpr uint32_t PANEL_Q = 64u * 128u;       // 64 rows x 128 B
     static constexpr uint32_t BLOCK_IL = 16384u;          // one 64 x 128 bf16 block (interleaved)
-    static constexpr uint32_t Q_BYTES = NP * PANEL_Q;
-    static constexpr uint32_t K_SLOT = NP * 128u * 128u;  // a tile: 128 rows
+    static constexpr uint32_t Q_BYTES = NPQ * PANEL_Q;
+    static constexpr uint32_t K_SLOT = NPQ * 128u * 128u; // a tile: 128 rows
     static constexpr uint32_t V_SLOT = 2u * 64u * 128u;   // a block; the PV MMA has M = 128 head-dim rows
     static constexpr uint32_t P_PANEL = 64u * 128u;       // 64 queries x 64 keys bf16
     static constexpr uint32_t P_BYTES = 4u * P_PANEL;     // a step: 256 keys
@@ -96,9 +101,10 @@ struct AttnLayout {
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + KSLOTS * K_SLOT;
     static constexpr uint32_t OFF_P = OFF_V + VSLOTS * V_SLOT;
-    static constexpr uint32_t OFF_AUX = OFF_P + 2 * P_BYTES;
+    static constexpr uint32_t OFF_SK = OFF_P + 2 * P_BYTES;  // e4m3: a step's key scales, per warpgroup, two steps
+    static constexpr uint32_t OFF_AUX = OFF_SK + (F8 ? 2u * 2u * 256u * 4u : 0u);
     // K tile (B operand of the S MMA, K-major): 8-row group stride and panel offset
-    static constexpr uint32_t K_SBO = IL ? 2048u : 1024u;
+    static constexpr uint32_t K_SBO = (IL && !F8) ? 2048u : 1024u;
     static constexpr uint32_t K_PANEL = IL ? 1024u : 128u * 128u;
     // V block (A operand of the PV MMA, MN-major): head-dim panel stride (LBO),
     // 8-row group stride (SBO), and the step between 16-key k-slices
@@ -106,9 +112,13 @@ struct AttnLayout {
     static constexpr uint32_t V_SBO = IL ? 2048u : 1024u;
     static constexpr uint32_t V_K16 = IL ? 4096u : 2048u;
     static_assert(!IL || D == 128, "interleaved layout is for head_dim 128");
+    static_assert(!F8 || D == 128, "the e4m3 path is for head_dim 128");
 };
 
+template <bool F8>
 struct AttnAux {
+    static constexpr int KSLOTS = Rings<F8>::K;
+    static constexpr int VSLOTS = Rings<F8>::V;
     uint64_t q_full;
     uint64_t k_full[KSLOTS], k_empty[KSLOTS];
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
@@ -124,12 +134,13 @@ struct AttnAux {
     int lst[LIST_SMEM];              // the CTA's block list (entries past LIST_SMEM stay in global memory)
 };
 
-static_assert(offsetof(AttnAux, alpha) % 16 == 0, "alpha is read with 16-byte loads");
+static_assert(offsetof(AttnAux<false>, alpha) % 16 == 0, "alpha is read with 16-byte loads");
+static_assert(offsetof(AttnAux<true>, alpha) % 16 == 0, "alpha is read with 16-byte loads");
 
-template <int D, bool IL>
+template <int D, bool IL, bool F8>
 constexpr uint32_t attn_smem_bytes()
 {
-    return AttnLayout<D, IL>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux)) + 1024u;
+    return AttnLayout<D, IL, F8>::OFF_AUX + static_cast<uint32_t>(sizeof(AttnAux<F8>)) + 1024u;
 }
 
 // Token rows of KV block g (0 when g is not a valid block id) and its first
@@ -198,17 +209,18 @@ __device__ __forceinline__ void tmem_ld128_nowait(uint32_t taddr, float (&v)[128
     }
 }
 
-template <int D, bool IL>
+template <int D, bool IL, bool F8>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rem,
             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k_rem,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_v_rem,
             const AttnArgs a)
 {
-    using L = AttnLayout<D, IL>;
+    using L = AttnLayout<D, IL, F8>;
+    constexpr int KSLOTS = L::KSLOTS, VSLOTS = L::VSLOTS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    AttnAux& x = *reinterpret_cast<AttnAux*>(smem + L::OFF_AUX);
+    AttnAux<F8>& x = *reinterpret_cast<AttnAux<F8>*>(smem + L::OFF_AUX);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the merge kernel of a split call may be scheduled once every CTA has started
@@ -292,8 +304,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (lane == 0) tma_prefetch_desc(&tm_k);
             __syncwarp();
             const CUtensorMap* mq = (q_rows == 64) ? &tm_q : &tm_q_rem;
-            mbar_arrive_expect_tx_elect(&x.q_full, static_cast<uint32_t>(L::NP * q_rows * 128));
-            for (int p = 0; p < L::NP; ++p)
+            mbar_arrive_expect_tx_elect(&x.q_full, static_cast<uint32_t>(L::NPQ * q_rows * 128));
+            for (int p = 0; p < L::NPQ; ++p)
                 tma_load_2d_elect(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
             int armed = 0;
             for (int t = 0; t < n_tiles; ++t) {
@@ -303,16 +315,23 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     rows[h] = block_rows(a, list_entry(x.lst, lst, 2 * t + h), bh, &first[h]);
                     if (rows[h] == 0 && lane == 0) record_error(a.err, DEVERR_LIST | 2);
                 }
-                const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NP);
+                const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NPQ);
                 const int s = t % KSLOTS;
                 if (!mbar_wait(&x.k_empty[s], ((t / KSLOTS) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
                 if (bytes) mbar_arrive_expect_tx_elect(&x.k_full[s], bytes);
                 else mbar_arrive_elect(&x.k_full[s]);
                 uint8_t* slot = smem + L::OFF_K + s * L::K_SLOT;
                 for (int h = 0; h < nb; ++h)
-                    if (rows[h])
-                        load_block<D, IL>(slot + h * (IL ? L::BLOCK_IL : 64u * 128u), 128u * 128u, rows[h], first[h],
-                                          &tm_k, &tm_k_rem, &x.k_full[s]);
+                    if (rows[h]) {
+                        if constexpr (F8) {
+                            // e4m3 rows are 128 bytes: one 2-D box per block, blocks 8 KB apart
+                            tma_load_2d_elect(slot + h * 8192u, rows[h] == 64 ? &tm_k : &tm_k_rem, 0, first[h],
+                                              &x.k_full[s]);
+                        } else {
+                            load_block<D, IL>(slot + h * (IL ? L::BLOCK_IL : 64u * 128u), 128u * 128u, rows[h],
+                                              first[h], &tm_k, &tm_k_rem, &x.k_full[s]);
+                        }
+                    }
                 armed = t + 1;
             }
             if (*abort_flag) {
@@ -352,7 +371,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // warp W_PV the PV MMAs; the waits below are normally already satisfied, which keeps
         // each issuing warp's code path short.
         {
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
+            constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(64, 128) : idesc_bf16_f32(64, 128, false, false);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, false);
             // A descriptor's start field is the byte address >> 4, so an operand at a byte
             // offset o from a base is the base descriptor + (o >> 4).
@@ -377,11 +396,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (!mbar_wait(&x.k_full[ks], (t / KSLOTS) & 1, abort_flag, a.err, 0x22)) return false;
                     const uint32_t d_addr = tmem + 128u * static_cast<uint32_t>(bsel) + (h ? (16u << 16) : 0u);
                     const uint64_t kb = dK + ((static_cast<uint32_t>(ks) * L::K_SLOT) >> 4);
+                    if constexpr (F8) {
+                        // e4m3: K = 32 per MMA, one 128-byte row per operand row
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t oq = ((kk >> 2) * L::PANEL_Q + (kk & 3) * 32) >> 4;
-                        const uint32_t ok_ = ((kk >> 2) * L::K_PANEL + (kk & 3) * 32) >> 4;
-                        umma_bf16_elect(d_addr, dQ + oq, kb + ok_, IDESC_S, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            umma_f8_elect(d_addr, dQ + ((kk * 32) >> 4), kb + ((kk * 32) >> 4), IDESC_S, kk > 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oq = ((kk >> 2) * L::PANEL_Q + (kk & 3) * 32) >> 4;
+                            const uint32_t ok_ = ((kk >> 2) * L::K_PANEL + (kk & 3) * 32) >> 4;
+                            umma_bf16_elect(d_addr, dQ + oq, kb + ok_, IDESC_S, kk > 0 ? 1u : 0u);
+                        }
                     }
                     umma_commit_elect(&x.k_empty[ks]);
                     issued_any = true;
@@ -432,11 +458,36 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int bar_id = 1 + g;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
         const uint32_t o_col = TM_O + 64u * static_cast<uint32_t>(g);
-        const float sl2 = a.scale_log2;
+        // Scores of the e4m3 path are S8 = <q8, k8>; the real score is S8 * s_q(row) * s_k(key),
+        // so the row's multiplier is scale * log2(e) * s_q(row) and each key's s_k comes per step.
+        float sl2 = a.scale_log2;
+        if constexpr (F8) sl2 = qr < q_rows ? sl2 * __ldg(a.q_scale + q_row0 + qr) : 0.f;
         // this thread's P row: panels 2*hh and 2*hh+1 (keys 128*hh ... 128*hh+127 of the step)
         uint8_t* prow = smem + L::OFF_P + g * L::P_BYTES + (2 * hh) * L::P_PANEL + qr * 128;
         float m_run = -INFINITY;  // stabiliser of this row (identical in lanes l and l^16)
         float l_run = 0.f;        // this thread's share of the row's softmax denominator
+
+        // e4m3: the key scales of this warpgroup's next step, fetched a step ahead (thread i of
+        // the warpgroup holds keys i and i + 128 of the step) so their L2 latency overlaps work
+        float kv_next[2] = {0.f, 0.f};
+        const int wg_i = (warp - W_SOFT0 - 4 * g) * 32 + lane;
+        auto fetch_scales = [&](int st) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int key = wg_i + 128 * half;
+                const int e = 2 * (2 * st + half) + ((key & 127) >> 6);
+                const int ri = key & 63;
+                float kv = 0.f;
+                if (e < cnt) {
+                    int first = 0;
+                    if (block_rows(a, list_entry(x.lst, lst, e), bh, &first) > ri) kv = __ldg(a.k_scale + first + ri);
+                }
+                kv_next[half] = kv;
+            }
+        };
+        if constexpr (F8) {
+            if (g < n_steps) fetch_scales(g);
+        }
 
         int j = 0;  // local step index of this warpgroup
         for (int s = g; s < n_steps; s += 2, ++j) {
@@ -444,12 +495,30 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int rows0 = entry_rows(a, x.lst, lst, 2 * tile, cnt);
             const int rows1 = entry_rows(a, x.lst, lst, 2 * tile + 1, cnt);
             const int bsel = s % SBUFS;
+            float* sk = nullptr;  // e4m3: this step's 256 key scales in shared memory
+            if constexpr (F8) {
+                // this step's scales (fetched a step ago) through shared memory to every thread
+                sk = reinterpret_cast<float*>(smem + L::OFF_SK) + (g * 2 + (j & 1)) * 256;
+                sk[wg_i] = kv_next[0];
+                sk[wg_i + 128] = kv_next[1];
+                named_bar_sync(bar_id, 128);
+                if (s + 2 < n_steps) fetch_scales(s + 2);
+            }
             mbar_wait(&x.s_full[bsel], (s / SBUFS) & 1, abort_flag, a.err, 0x30);
             __syncwarp();
             tc_fence_after();
             float sv[128];
             tmem_ld128_nowait(lane_base + 128u * bsel, sv);
             tmem_ld_wait();
+            if constexpr (F8) {
+                const float* skh = sk + 128 * hh;
+#pragma unroll
+                for (int c = 0; c < 128; c += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(skh + c);
+                    fmul2(sv[c], sv[c + 1], t4.x, t4.y);
+                    fmul2(sv[c + 2], sv[c + 3], t4.z, t4.w);
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&x.s_free[bsel]);
@@ -694,23 +763,23 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a)
     }
 }
 
-template <int D, bool IL>
-cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, int n_rows, cudaStream_t s)
+template <int D, bool IL, bool F8>
+cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t s)
 {
-    constexpr uint32_t smem = attn_smem_bytes<D, IL>();
+    constexpr uint32_t smem = attn_smem_bytes<D, IL, F8>();
     static_assert(smem <= 232448, "shared memory plan exceeds 227 KB");
     static int configured_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(attn_kernel<D, IL>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = cudaFuncSetAttribute(attn_kernel<D, IL, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    const int tail = a.pieces > 0 ? n_rows - a.n_whole : 0;
-    const long long grid = a.pieces > 0 ? a.n_whole + static_cast<long long>(tail) * a.pieces : n_rows;
-    attn_kernel<D, IL><<<static_cast<unsigned>(grid), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
+    const int tail = a.pieces > 0 ? a.n_rows - a.n_whole : 0;
+    const long long grid = a.n_units;
+    attn_kernel<D, IL, F8><<<static_cast<unsigned>(grid), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
                                                                              m.v_rem, a);
     e = cudaGetLastError();
     if (e != cudaSuccess || tail == 0) return e;
@@ -729,12 +798,18 @@ cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, int n_rows, cuda
 
 }  // namespace
 
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s)
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, cudaStream_t s)
 {
-    if (n_rows <= 0) return cudaSuccess;
+    if (a.n_units <= 0) return cudaSuccess;
     if (D == 128)
-        return interleaved ? launch_attn_t<128, true>(m, a, n_rows, s) : launch_attn_t<128, false>(m, a, n_rows, s);
-    return launch_attn_t<64, false>(m, a, n_rows, s);
+        return interleaved ? launch_attn_t<128, true, false>(m, a, s) : launch_attn_t<128, false, false>(m, a, s);
+    return launch_attn_t<64, false, false>(m, a, s);
+}
+
+cudaError_t launch_attn_fp8(const AttnMaps& m, const AttnArgs& a, bool v_interleaved, cudaStream_t s)
+{
+    if (a.n_units <= 0) return cudaSuccess;
+    return v_interleaved ? launch_attn_t<128, true, true>(m, a, s) : launch_attn_t<128, false, true>(m, a, s);
 }
 
 }  // namespace lf

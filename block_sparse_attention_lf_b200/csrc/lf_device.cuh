@@ -227,6 +227,20 @@ __device__ __forceinline__ void umma_bf16_elect(uint32_t d_tmem, uint64_t adesc,
         : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc], e4m3 inputs (kind::f8f6f4, K = 32 per
+// MMA), fp32 accumulate, issued by one elected lane of the converged calling warp.
+__device__ __forceinline__ void umma_f8_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by the elected
 // lane has completed (called by the converged warp that issued them; the
 // elected lane is the same one umma_bf16_elect picks).
@@ -315,6 +329,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f8f6f4 with e4m3 A/B (both K-major) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                                   // D format: f32
+           | (0u << 7)                                 // A format: e4m3
+           | (0u << 10)                                // B format: e4m3
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 // ---- named barriers --------------------------------------------------------
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {
@@ -349,6 +373,18 @@ __device__ __forceinline__ void ffma2_bc(float& d0, float& d1, float a0, float a
         "mov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d0), "=f"(d1)
         : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (a0, a1) *= (b0, b1) as one packed f32x2 multiply.
+__device__ __forceinline__ void fmul2(float& a0, float& a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%0, %1};\n\t"
+        "mov.b64 rb, {%2, %3};\n\t"
+        "mul.rn.f32x2 ra, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, ra;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1));
 }
 
 // (s0, s1) += (a0, a1) as one packed f32x2 add.

@@ -18,6 +18,7 @@ struct PoolArgs {
     long long kv_stride;  // tokens between heads in k
     int f0, nk;           // KV frames [f0, f0 + nk) are pooled
     int pool_q;           // also pool the query frames
+    int* err;             // device error word (an expired bounded wait)
 };
 
 struct SelectFramesArgs {
@@ -47,7 +48,7 @@ struct SelectBlocks1dArgs {
     int BH, D, Rq, Nkv, kb, list_cap, chunk_index;
 };
 
-constexpr int SEL1D_MAX_NKV = 16384;  // candidate keys held in shared memory (128 KB)
+constexpr int SEL1D_MAX_NKV = 16384;  // candidate scores held in shared memory (64 KB per scored row)
 
 // Coarse frame retrieval: a k-means index over each head's memory-frame means.
 constexpr int IVF_MAX_CLUSTERS = 64;
@@ -82,13 +83,17 @@ struct AttnArgs {
     long long kv_stride;
     float scale_log2;  // softmax scale * log2(e)
     int* err;
-    // Split of the last, partial wave: query blocks [0, n_whole) take one CTA
-    // each; every later query block's list is cut into `pieces` consecutive
-    // pieces, one CTA each, whose normalised fp32 partial rows and (max, sum)
-    // pairs go to part_o / part_ml and are merged by a second kernel.
+    // Split of the tail: query blocks [0, n_whole) are one work unit each; every
+    // later query block's list is cut into `pieces` consecutive pieces, one unit
+    // each, whose normalised fp32 partial rows and (stabiliser, sum) pairs go to
+    // part_o / part_ml and are merged by a second kernel.
     int n_whole, pieces;  // pieces == 0: no split
     float* part_o;        // [slot][64][D]; slot = (query block - n_whole) * pieces + piece
-    float* part_ml;       // [slot][64][2]: max of scale*log2(e)*score, softmax denominator
+    float* part_ml;       // [slot][64][2]: stabiliser (log2 units), softmax denominator
+    int n_rows;           // query blocks of the call (B * H * Rq)
+    int n_units;          // CTAs of the attention grid: n_whole whole lists + (n_rows - n_whole) * pieces pieces
+    const float* q_scale;  // e4m3 path: per-token scales of q8 [B*H*Lq] and k8 [B*H*kv_stride]
+    const float* k_scale;
 };
 
 struct AttnMaps {
@@ -98,10 +103,17 @@ struct AttnMaps {
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s);
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s);
+// both selection levels in one launch (frame_sel and the block lists, as the two above)
+cudaError_t launch_select_fused(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s);
+// per-row e4m3 codes and fp32 scales of n_rows rows of D bf16 values
+cudaError_t launch_quant_rows(const uint16_t* x, long long n_rows, int D, uint8_t* x8, float* scale, cudaStream_t s);
 cudaError_t launch_select_blocks_1d(const SelectBlocks1dArgs& a, cudaStream_t s);
 cudaError_t launch_frame_index(const FrameIndexArgs& a, cudaStream_t s);
 cudaError_t launch_select_frames_ivf(const SelectFramesIvfArgs& a, cudaStream_t s);
 // interleaved: K/V tensor maps are the 4-D block maps (head_dim 128 only).
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, int n_rows, cudaStream_t s);
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, int D, bool interleaved, cudaStream_t s);
+// e4m3 q/k (head_dim 128): maps q / q_rem / k / k_rem are uint8 row maps, v / v_rem bf16
+// (4-D block maps when v_interleaved)
+cudaError_t launch_attn_fp8(const AttnMaps& m, const AttnArgs& a, bool v_interleaved, cudaStream_t s);
 
 }  // namespace lf

@@ -29,26 +29,25 @@ namespace {
 
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
+constexpr int SEL_FUSED_MAX_WARPS = 16;
 
-// KPL = key slots per lane = ceil(n_mem / 32).
+// T_r of scored row `row` (one warp): frame scores of the memory frames, top-k_f by
+// warp arg-max rounds, forced frames added; written ascending to out (global) and, when
+// sel_copy is not NULL, to sel_copy too. KPL = key slots per lane = ceil(n_mem / 32).
 template <int D, int KPL>
-__global__ void __launch_bounds__(SEL_THREADS) select_frames_kernel(const SelectFramesArgs a)
+__device__ __forceinline__ void frames_of_row(const SelectFramesArgs& a, long long row, int lane, const float (&qv)[D / 32],
+                                              int* out, int* sel_copy)
 {
-    constexpr int EPL = D / 32;
-    const int lane = threadIdx.x & 31;
-    const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
-    if (row >= static_cast<long long>(a.BH) * a.Rq) return;
-    int* out = a.frame_sel + row * a.n_sel;
     if (a.chunk_index == 1) {
-        for (int t = lane; t < a.NF; t += 32) out[t] = t;
+        for (int t = lane; t < a.NF; t += 32) {
+            out[t] = t;
+            if (sel_copy) sel_copy[t] = t;
+        }
         return;
     }
     const int bh = static_cast<int>(row / a.Rq);
     const int n_mem = a.NF - a.n_sink - a.n_recent - a.n_cur;
     const int kf = a.topk < n_mem ? a.topk : n_mem;
-
-    float qv[EPL];
-    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
     const float* kmem = a.k_frame + (static_cast<long long>(bh) * a.NF + a.n_sink) * D;
 
     uint64_t key[KPL];
@@ -74,44 +73,56 @@ __global__ void __launch_bounds__(SEL_THREADS) select_frames_kernel(const Select
     }
 
     // T_r = sinks, selected memory frames (ascending), recent + current frames.
-    for (int t = lane; t < a.n_sink; t += 32) out[t] = t;
+    for (int t = lane; t < a.n_sink; t += 32) {
+        out[t] = t;
+        if (sel_copy) sel_copy[t] = t;
+    }
     int prefix = a.n_sink;
     const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
     for (int i = 0; i < KPL; ++i) {
         const bool s = (sel >> i) & 1u;
         const uint32_t mask = __ballot_sync(0xffffffffu, s);
-        if (s) out[prefix + __popc(mask & lt)] = a.n_sink + i * 32 + lane;
+        if (s) {
+            out[prefix + __popc(mask & lt)] = a.n_sink + i * 32 + lane;
+            if (sel_copy) sel_copy[prefix + __popc(mask & lt)] = a.n_sink + i * 32 + lane;
+        }
         prefix += __popc(mask);
     }
     const int tail0 = a.NF - a.n_recent - a.n_cur;
-    for (int t = lane; t < a.n_recent + a.n_cur; t += 32) out[a.n_sink + kf + t] = tail0 + t;
+    for (int t = lane; t < a.n_recent + a.n_cur; t += 32) {
+        out[a.n_sink + kf + t] = tail0 + t;
+        if (sel_copy) sel_copy[a.n_sink + kf + t] = tail0 + t;
+    }
 }
 
-// One warp per (row, selected-frame slot). KPL = ceil(bpf / 32).
 template <int D, int KPL>
-__global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const SelectBlocksArgs a)
+__global__ void __launch_bounds__(SEL_THREADS) select_frames_kernel(const SelectFramesArgs a)
 {
     constexpr int EPL = D / 32;
     const int lane = threadIdx.x & 31;
-    const long long gw = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
-    if (gw >= static_cast<long long>(a.BH) * a.Rq * a.n_sel) return;
-    const long long row = gw / a.n_sel;
-    const int s = static_cast<int>(gw - row * a.n_sel);
+    const long long row = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
+    if (row >= static_cast<long long>(a.BH) * a.Rq) return;
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    frames_of_row<D, KPL>(a, row, lane, qv, a.frame_sel + row * a.n_sel, nullptr);
+}
+
+// The top-k_b blocks of selected frame slot s (frame tau) of scored row `row` (one
+// warp), written ascending into the row's list at s * k_b. KPL = ceil(bpf / 32).
+template <int D, int KPL>
+__device__ __forceinline__ void blocks_of_frame(const SelectBlocksArgs& a, long long row, int s, int tau, int lane,
+                                                const float (&qv)[D / 32])
+{
     const int bh = static_cast<int>(row / a.Rq);
     int* out = a.block_list + row * a.list_cap + static_cast<long long>(s) * a.kb;
     if (s == 0 && lane == 0) a.block_count[row] = a.n_sel * a.kb;
-
-    const int tau = (a.chunk_index == 1) ? s : __ldg(a.frame_sel + row * a.n_sel + s);
     if (tau < 0 || tau >= a.NF) {
         // A frame id outside the call: write ids the attention kernel rejects.
         for (int t = lane; t < a.kb; t += 32) out[t] = -1;
         if (lane == 0) record_error(a.err, DEVERR_LIST | 3);
         return;
     }
-
-    float qv[EPL];
-    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
     const float* kblk = a.k_pool + (static_cast<long long>(bh) * a.NF * a.bpf + static_cast<long long>(tau) * a.bpf) * D;
 
     uint64_t key[KPL];
@@ -145,86 +156,118 @@ __global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const Select
     }
 }
 
+// One warp per (row, selected-frame slot).
+template <int D, int KPL>
+__global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const SelectBlocksArgs a)
+{
+    constexpr int EPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long gw = static_cast<long long>(blockIdx.x) * SEL_WARPS + (threadIdx.x >> 5);
+    if (gw >= static_cast<long long>(a.BH) * a.Rq * a.n_sel) return;
+    const long long row = gw / a.n_sel;
+    const int s = static_cast<int>(gw - row * a.n_sel);
+    const int tau = (a.chunk_index == 1) ? s : __ldg(a.frame_sel + row * a.n_sel + s);
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    blocks_of_frame<D, KPL>(a, row, s, tau, lane, qv);
+}
+
+// Both levels for one scored row per CTA, in one launch: warp 0 picks T_r (to frame_sel
+// and to shared memory), then warp w takes the blocks of selected frames w, w + W, ...
+// The arithmetic is the two kernels' above, so the result is bit-identical to
+// select_frames_kernel followed by select_blocks_kernel; the second launch and its
+// dependent gap are gone.
+template <int D, int KPLF, int KPLB>
+__global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(const SelectFramesArgs fa,
+                                                                                const SelectBlocksArgs ba)
+{
+    constexpr int EPL = D / 32;
+    extern __shared__ int sel_s[];  // [n_sel]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+    const long long row = blockIdx.x;
+    float qv[EPL];
+    load_lane<EPL>(qv, fa.q_pool + row * D + lane * EPL);
+    if (warp == 0) frames_of_row<D, KPLF>(fa, row, lane, qv, fa.frame_sel + row * fa.n_sel, sel_s);
+    __syncthreads();
+    for (int s = warp; s < ba.n_sel; s += n_warps) blocks_of_frame<D, KPLB>(ba, row, s, sel_s[s], lane, qv);
+}
+
 // One-dimensional selection (the single-granularity variant of the ablation in
-// "南洋理工大学打造视频生成新引擎", 163.com, section 4): one CTA per scored row,
-// every KV block of the head a candidate. Warps score groups of 32 candidates
-// into 64-bit keys in shared memory; the kb-th largest key T is built bit by
-// bit from the top (a candidate bit stays when at least kb keys are >= the
-// value with it set; keys are unique, so exactly kb keys are >= T); a ballot
-// compaction in index order writes the kept ids ascending.
+// "南洋理工大学打造视频生成新引擎", 163.com, section 4): every KV block of the head is a
+// candidate. One CTA per scored row: its warps score groups of 32 candidates into 32-bit
+// orderable scores in shared memory; then one warp finds the exact score T of the kb-th
+// largest bit by bit from the top (32 rounds of warp ballot counts, no block barrier) and
+// writes, in index order, every candidate scoring above T and the lowest-indexed ones
+// scoring exactly T until kb are kept: the order of the two-level kernels' 64-bit keys
+// (score, then lower index), so the lists are those of a full sort.
 template <int D>
 __global__ void __launch_bounds__(SEL_THREADS) select_blocks_1d_kernel(const SelectBlocks1dArgs a)
 {
     constexpr int EPL = D / 32;
-    extern __shared__ uint64_t keys[];  // [Nkv]
-    __shared__ int red[2][SEL_WARPS];   // per-warp partial counts, two alternating slots
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    extern __shared__ uint32_t sc[];  // [Nkv] orderable scores
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long row = blockIdx.x;
-    const int bh = static_cast<int>(row / a.Rq);
     const int n = a.Nkv;
+    const int bh = static_cast<int>(row / a.Rq);
     int* out = a.block_list + row * a.list_cap;
     const int keep = (a.chunk_index == 1 || a.kb >= n) ? n : a.kb;
-    if (tid == 0) a.block_count[row] = keep;
+    if (threadIdx.x == 0) a.block_count[row] = keep;
     if (keep == n) {
-        for (int g = tid; g < n; g += SEL_THREADS) out[g] = g;
+        for (int g = threadIdx.x; g < n; g += SEL_THREADS) out[g] = g;
         return;
     }
     float qv[EPL];
     load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
     const float* kblk = a.k_pool + static_cast<long long>(bh) * n * D;
     for (int grp = warp; grp * 32 < n; grp += SEL_WARPS) {
-        const float sc = score_group<D>(qv, kblk, grp * 32, n, lane);
-        const int g = grp * 32 + lane;
-        if (g < n) keys[g] = make_key(sc, g);
+        const float s = score_group<D>(qv, kblk, grp * 32, n, lane);
+        if (grp * 32 + lane < n) sc[grp * 32 + lane] = orderable(s);
     }
     __syncthreads();
-    uint64_t T = 0;
-    for (int bit = 63; bit >= 0; --bit) {
-        const uint64_t cand = T | (1ull << bit);
-        unsigned c = 0;
-        for (int g = tid; g < n; g += SEL_THREADS) c += keys[g] >= cand ? 1u : 0u;
-        c = __reduce_add_sync(0xffffffffu, c);
-        const int buf = bit & 1;
-        if (lane == 0) red[buf][warp] = static_cast<int>(c);
-        __syncthreads();
-        int total = 0;
-#pragma unroll
-        for (int w = 0; w < SEL_WARPS; ++w) total += red[buf][w];
-        if (total >= keep) T = cand;
-    }
-    __syncthreads();  // the last round's counts are read before the slots are reused
-    int prefix = 0;
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int base = 0, it = 0; base < n; base += SEL_THREADS, ++it) {
-        const int g = base + tid;
-        const bool sel = g < n && keys[g] >= T;
-        const uint32_t m = __ballot_sync(0xffffffffu, sel);
-        const int buf = it & 1;
-        if (lane == 0) red[buf][warp] = __popc(m);
-        __syncthreads();
-        int before = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < SEL_WARPS; ++w) {
-            const int v = red[buf][w];
-            total += v;
-            before += (w < warp) ? v : 0;
+    if (warp != 0) return;
+    // T = the largest 32-bit value with at least `keep` scores >= T, built bit by bit
+    uint32_t prefix = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = prefix | (1u << bit);
+        int c = 0;
+        for (int base = 0; base < n; base += 32) {
+            const int g = base + lane;
+            c += __popc(__ballot_sync(0xffffffffu, g < n && sc[g] >= cand));
         }
-        if (sel) out[prefix + before + __popc(m & lt)] = g;
-        prefix += total;
+        if (c >= keep) prefix = cand;
+    }
+    int above = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int g = base + lane;
+        above += __popc(__ballot_sync(0xffffffffu, g < n && sc[g] > prefix));
+    }
+    const int need = keep - above;  // scores equal to T still to take, lowest index first
+    int pos = 0, eq_seen = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += 32) {
+        const int g = base + lane;
+        const uint32_t v = g < n ? sc[g] : 0u;
+        const bool eq = g < n && v == prefix;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool take = (g < n && v > prefix) || (eq && eq_seen + __popc(eqm & lt) < need);
+        const uint32_t tm = __ballot_sync(0xffffffffu, take);
+        if (take) out[pos + __popc(tm & lt)] = g;
+        pos += __popc(tm);
+        eq_seen += __popc(eqm);
     }
 }
 
 template <int D>
 cudaError_t launch_blocks_1d_d(const SelectBlocks1dArgs& a, cudaStream_t s)
 {
-    const size_t smem = static_cast<size_t>(a.Nkv) * sizeof(uint64_t);
+    const size_t smem = static_cast<size_t>(a.Nkv) * sizeof(uint32_t);
     static int configured_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
         e = cudaFuncSetAttribute(select_blocks_1d_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(SEL1D_MAX_NKV * sizeof(uint64_t)));
+                                 static_cast<int>(SEL1D_MAX_NKV * sizeof(uint32_t)));
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
@@ -257,6 +300,37 @@ cudaError_t launch_blocks_d(const SelectBlocksArgs& a, unsigned grid, cudaStream
     return cudaGetLastError();
 }
 
+template <int D, int KPLF, int KPLB>
+cudaError_t launch_fused_k(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s)
+{
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(fa.BH) * fa.Rq);
+    const int warps = ba.n_sel < SEL_FUSED_MAX_WARPS ? ba.n_sel : SEL_FUSED_MAX_WARPS;
+    select_fused_kernel<D, KPLF, KPLB><<<grid, 32 * warps, static_cast<size_t>(fa.n_sel) * sizeof(int), s>>>(fa, ba);
+    return cudaGetLastError();
+}
+
+template <int D, int KPLF>
+cudaError_t launch_fused_b(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s)
+{
+    const int kpl = (ba.bpf + 31) / 32;
+    if (kpl <= 1) return launch_fused_k<D, KPLF, 1>(fa, ba, s);
+    if (kpl <= 2) return launch_fused_k<D, KPLF, 2>(fa, ba, s);
+    return launch_fused_k<D, KPLF, 4>(fa, ba, s);
+}
+
+template <int D>
+cudaError_t launch_fused_d(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s)
+{
+    const int n_mem = fa.NF - fa.n_sink - fa.n_recent - fa.n_cur;
+    const int kpl = (n_mem + 31) / 32;
+    if (fa.chunk_index == 1 || kpl <= 1) return launch_fused_b<D, 1>(fa, ba, s);
+    if (kpl <= 2) return launch_fused_b<D, 2>(fa, ba, s);
+    if (kpl <= 4) return launch_fused_b<D, 4>(fa, ba, s);
+    if (kpl <= 8) return launch_fused_b<D, 8>(fa, ba, s);
+    if (kpl <= 16) return launch_fused_b<D, 16>(fa, ba, s);
+    return launch_fused_b<D, 32>(fa, ba, s);
+}
+
 }  // namespace
 
 cudaError_t launch_select_blocks_1d(const SelectBlocks1dArgs& a, cudaStream_t s)
@@ -271,6 +345,12 @@ cudaError_t launch_select_frames(const SelectFramesArgs& a, cudaStream_t s)
     if (rows <= 0) return cudaSuccess;
     const unsigned grid = static_cast<unsigned>((rows + SEL_WARPS - 1) / SEL_WARPS);
     return a.D == 128 ? launch_frames_d<128>(a, grid, s) : launch_frames_d<64>(a, grid, s);
+}
+
+cudaError_t launch_select_fused(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s)
+{
+    if (static_cast<long long>(fa.BH) * fa.Rq <= 0) return cudaSuccess;
+    return fa.D == 128 ? launch_fused_d<128>(fa, ba, s) : launch_fused_d<64>(fa, ba, s);
 }
 
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t s)

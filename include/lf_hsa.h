@@ -14,6 +14,7 @@
  *                        plus the always-kept sink / recent / current frames
  *   lf_select_blocks     per selected frame: block scores, top-k blocks J_r(tau),
  *                        written as a compacted block list (the mask B_r)
+ *   lf_select_mask       both selection levels in one launch
  *   lf_select_blocks_1d  one-dimensional variant: global block top-k over all
  *                        KV blocks, no frame level (the ablation baseline)
  *   lf_frame_index_build / lf_select_frames_ivf  coarse frame retrieval: a
@@ -26,6 +27,8 @@
  *   lf_attn_split_plan   that split's plan and workspace size (host only)
  *   lf_block_sparse_attn_static  the split attention for callers that cannot
  *                        allocate: its scratch is an array inside the library
+ *   lf_quant_fp8_rows    per-token e4m3 codes and scales (the FP8 attention's q, k)
+ *   lf_block_sparse_attn_fp8  the attention with e4m3 q and k (tcgen05 kind::f8f6f4)
  *
  * plus the host-side Chunk-Aware Growth budget solver (same pages, stage 1 /
  * Technical Summary 2.1).
@@ -195,6 +198,18 @@ LF_API lf_status lf_select_blocks(const lf_hsa_shape* shape, int32_t chunk_index
                            int32_t list_cap, void* stream);
 
 /*
+ * Both levels of the mask selection in one launch: lf_select_frames followed by
+ * lf_select_blocks (same passages, arguments, layouts and errors), computed per
+ * query block by one CTA (frames, then the blocks of the selected frames) with
+ * the same arithmetic, so frame_sel, block_list and block_count are
+ * bit-identical to the two separate calls.
+ */
+LF_API lf_status lf_select_mask(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_frames,
+                         int32_t topk_blocks, const float* q_pool, const float* k_frame,
+                         const float* k_pool, int32_t* frame_sel, int32_t* block_list,
+                         int32_t* block_count, int32_t list_cap, void* stream);
+
+/*
  * One-dimensional (single-granularity) block selection: the variant without
  * the frame level that the ablation of "南洋理工大学打造视频生成新引擎"
  * (163.com, section 4) compares against. Reading (the pages name the variant
@@ -259,6 +274,24 @@ LF_API lf_status lf_select_frames_ivf(const lf_hsa_shape* shape, int32_t chunk_i
                                int32_t n_clusters, int32_t n_probe, const float* q_pool,
                                const float* k_frame, const float* centroids, const int32_t* offsets,
                                const int32_t* members, int32_t* frame_sel, void* stream);
+
+/*
+ * Per-token e4m3 quantisation for the FP8 attention (lf_block_sparse_attn_fp8).
+ * The pages put FP8 with per-token activation scales on the model's linear
+ * layers ("南洋理工大学打造视频生成新引擎", 163.com, deployment section;
+ * gist.science, Technical Summary 4) and describe no FP8 attention; reading taken
+ * here: Q and K quantised per token (one scale per row of head_dim values).
+ *   x       [n_rows, head_dim] bf16 (e.g. q, or k with its head stride padding)
+ *   x8      [n_rows, head_dim] uint8 out: e4m3 codes (OCP E4M3: bias 7, 3 mantissa
+ *           bits, largest finite 448)
+ *   scales  [n_rows] fp32 out: s = fl32(amax / 448) (1 for an all-zero row)
+ * code = e4m3(fl32(x / s)) with IEEE fp32 division, round to nearest even,
+ * saturating at 448; x is about s * code. One warp per row.
+ * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_ARG (head_dim not 64 or 128, n_rows
+ * < 0), LF_ERR_SHAPE, LF_ERR_CUDA.
+ */
+LF_API lf_status lf_quant_fp8_rows(const uint16_t* x, int64_t n_rows, int32_t head_dim, uint8_t* x8,
+                            float* scales, void* stream);
 
 /*
  * Block-sparse softmax attention (paper.rainbus.top, execution flow, stage 3,
@@ -359,6 +392,24 @@ LF_API lf_status lf_block_sparse_attn_static(const lf_hsa_shape* shape, const ui
                                       const int32_t* block_count, int32_t list_cap,
                                       float softmax_scale, uint16_t* out, int32_t tail_pieces,
                                       void* stream);
+
+/*
+ * Block-sparse attention with e4m3 queries and keys (head_dim 128): the FP8
+ * attention of this library. Same passage and mask as lf_block_sparse_attn; the
+ * FP8 reading is lf_quant_fp8_rows'. Scores are <q8, k8> (exact e4m3 products,
+ * fp32 accumulation on the tensor cores, kind::f8f6f4) times q_scale(row) *
+ * k_scale(key); the softmax is fp32 as in the bf16 path and P and V stay bf16.
+ *   q8       [B,H,Lq,128] uint8 e4m3 codes, q_scale [B,H,Lq] fp32
+ *   k8       [B,H,kv_stride,128] uint8 e4m3 codes, k_scale [B,H,kv_stride] fp32
+ *   v        [B,H,kv_stride,128] bf16
+ *   the rest as lf_block_sparse_attn_ws (list, scale, out, split and workspace).
+ * Errors: those of lf_block_sparse_attn_ws; LF_ERR_SHAPE when head_dim != 128.
+ */
+LF_API lf_status lf_block_sparse_attn_fp8(const lf_hsa_shape* shape, const uint8_t* q8, const uint8_t* k8,
+                                   const float* q_scale, const float* k_scale, const uint16_t* v,
+                                   const int32_t* block_list, const int32_t* block_count, int32_t list_cap,
+                                   float softmax_scale, uint16_t* out, int32_t tail_pieces,
+                                   void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
  * Chunk-Aware Growth budget solver, host only, fp64 (paper.rainbus.top,

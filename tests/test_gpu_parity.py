@@ -240,3 +240,38 @@ def test_split_matches_unsplit_layer480p():
     np.testing.assert_array_equal(oa[:first_tail_row], ob[:first_tail_row])
     d = np.abs(oa[first_tail_row:] - ob[first_tail_row:]).max()
     assert d <= parity.OUT_MAX_ABS, d
+
+
+@pytest.mark.parametrize("name,chunk", [("ragged_d128", 2), ("ragged_d64_odd_lists", 2), ("dense_first_chunk", 1),
+                                        ("no_memory_frames", 2), ("layer480p", 2), ("longvideo480p", 2)])
+def test_fused_selection_equals_two_kernels(name, chunk):
+    """lf_select_mask (both levels in one launch) writes exactly what lf_select_frames followed by
+    lf_select_blocks write: same frame rows, lists and counts, bit for bit."""
+    import block_sparse_attention_lf_b200 as L
+    if name in lf_synth.CONFIGS:
+        w = lf_synth.CONFIGS[name]
+        q, k, v = lf_synth.make_qkv(w)
+        ls = L.shape_from_workload(w)
+        kf = w.topk_frames
+        n_sel = L.lf_frames_selected(ls, chunk, kf)
+        kb = w.topk_blocks or L.lf_blocks_for_sparsity(w.sparsity, ls.Nkv, n_sel, ls.bpf)
+    else:
+        case = next(c for c in SMALL if c[0] == name)
+        _, B, H, D, F, (ns, nm, nr, nc), _, kf, kb, kscale, _ = case
+        ls = L.LfShape.make(B, H, D, F, ns + nm + nr + nc, ns, nr, nc)
+        q, k, v = _rand(zlib.crc32(name.encode()) % 1000, B, H, nc * F, ls.n_frames * F, D, kscale)
+    call = L.HSACall(ls, chunk, kf, kb)
+    b = call.buf
+    call.pool(q.cuda(), k.cuda())
+    fs2, bl2, bc2 = torch.full_like(b.frame_sel, -5), torch.full_like(b.block_list, -5), torch.full_like(b.block_count, -5)
+    L.lf_select_frames(ls, chunk, kf, b.q_pool, b.k_frame, fs2)
+    L.lf_select_blocks(ls, chunk, kf, kb, b.q_pool, b.k_pool, fs2, bl2, bc2, b.list_cap)
+    b.frame_sel.fill_(-9)
+    b.block_list.fill_(-9)
+    b.block_count.fill_(-9)
+    call.select()
+    torch.cuda.synchronize()
+    assert L.lf_get_device_error()[0] == 0
+    assert torch.equal(b.frame_sel, fs2) and torch.equal(b.block_count, bc2)
+    cnt = int(bc2.max())
+    assert torch.equal(b.block_list[..., :cnt], bl2[..., :cnt])
