@@ -494,6 +494,96 @@ def one_dim_report(L, lf_synth, peaks, steps, flush):
             "attn_frac_of_bf16_peak": round(flops / (att * 1e-6) / 1e12 / peaks["bf16"], 4)}
 
 
+def _time_us(fn, steps, flush, stream):
+    import torch
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.mean(ts)
+
+
+def fp8_report(L, lf_synth, peaks, steps, flush):
+    """layer480p through the FP8 attention (e4m3 q and k per token, bf16 softmax weights
+    and v) on the bf16 call's lists. Its roofline peak mixes the two rates: QK^T runs on
+    e4m3 tensor cores (the nominal 2x of bf16) and PV on bf16 ones, half the FLOPs each,
+    so the time at peak is F/2/(2P) + F/2/P and the effective peak 4P/3 (P = the measured
+    bf16 peak). k is quantised once per chunk (past frames do not change while a chunk
+    denoises), q per call: both are reported."""
+    import torch
+    w = lf_synth.CONFIGS["layer480p"]
+    shape = L.shape_from_workload(w)
+    kb = _kb(L, shape, w)
+    q, k, v = (t.cuda() for t in lf_synth.make_qkv(w))
+    call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb)
+    call(q, k, v)
+    b = call.buf
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device="cuda")
+    qs = torch.empty(q.shape[:-1], dtype=torch.float32, device="cuda")
+    ks = torch.empty(k.shape[:-1], dtype=torch.float32, device="cuda")
+    out8 = torch.empty_like(b.out)
+    stream = torch.cuda.current_stream()
+    quant_q = lambda: L.lf_quant_fp8_rows(q, q8, qs)
+    quant_k = lambda: L.lf_quant_fp8_rows(k, k8, ks)
+    attn8 = lambda: L.lf_block_sparse_attn_fp8(shape, q8, k8, qs, ks, v, b.block_list, b.block_count, b.list_cap,
+                                               0.0, out8, call.workspace, call.tail_pieces)
+    for _ in range(3):
+        quant_q(); quant_k(); attn8()
+    torch.cuda.synchronize()
+    st, detail = L.lf_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error: {st} {detail:#x}")
+    flops = credited_flops(b.block_list.cpu().numpy(), b.block_count.cpu().numpy(), shape.frame_tokens,
+                           shape.bpf, shape.head_dim, shape.n_cur)
+    t_q, t_k, t_a = (_time_us(f, steps, flush, stream) for f in (quant_q, quant_k, attn8))
+    t_bf16 = _time_us(lambda: call.attend(q, k, v), steps, flush, stream)
+    tf = flops / (t_a * 1e-6) / 1e12
+    mixed_peak = peaks["bf16"] * 4.0 / 3.0
+    return {"attn_fp8_us": round(t_a, 2), "attn_bf16_us_same_run": round(t_bf16, 2),
+            "quant_q_us": round(t_q, 2), "quant_k_us_once_per_chunk": round(t_k, 2),
+            "attn_fp8_tflops": round(tf, 1), "mixed_peak_tflops": round(mixed_peak, 1),
+            "attn_fp8_frac_of_mixed_peak": round(tf / mixed_peak, 4),
+            "quant_q_gbs": round((q.numel() * 3 + qs.numel() * 4) / (t_q * 1e-6) / 1e9, 1)}
+
+
+def ivf_report(L, lf_synth, peaks, steps, flush, n_clusters=8, n_probe=2):
+    """longvideo480p (60 memory frames) with the coarse frame index: index build (k-means
+    over the frame means, once per appended chunk), probed frame selection against the
+    exact one, and the recall of the exact top-k memory frames."""
+    import torch
+    w = lf_synth.CONFIGS["longvideo480p"]
+    shape = L.shape_from_workload(w)
+    kb = _kb(L, shape, w)
+    q, k, v = (t.cuda() for t in lf_synth.make_qkv(w))
+    call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb)
+    call.pool(q, k)
+    b = call.buf
+    idx = L.FrameIndex.empty(shape, n_clusters)
+    sel_ivf = torch.empty_like(b.frame_sel)
+    stream = torch.cuda.current_stream()
+    build = lambda: L.lf_frame_index_build(shape, b.k_frame, idx, iters=25)
+    probe = lambda: L.lf_select_frames_ivf(shape, w.chunk_index, w.topk_frames, idx, n_probe, b.q_pool,
+                                           b.k_frame, sel_ivf)
+    exact = lambda: L.lf_select_frames(shape, w.chunk_index, w.topk_frames, b.q_pool, b.k_frame, b.frame_sel)
+    for _ in range(3):
+        build(); probe(); exact()
+    torch.cuda.synchronize()
+    t_b, t_p, t_e = (_time_us(f, steps, flush, stream) for f in (build, probe, exact))
+    n_sink, n_mem = shape.n_sink, shape.n_frames - shape.n_sink - shape.n_recent - shape.n_cur
+    mem = lambda t: [set(f for f in r if n_sink <= f < n_sink + n_mem) for r in t.reshape(-1, t.shape[-1]).tolist()]
+    a_, e_ = mem(sel_ivf.cpu()), mem(b.frame_sel.cpu())
+    recall = sum(len(x & y) for x, y in zip(a_, e_)) / max(1, sum(len(y) for y in e_))
+    return {"n_clusters": n_clusters, "n_probe": n_probe, "index_build_us": round(t_b, 2),
+            "select_frames_ivf_us": round(t_p, 2), "select_frames_exact_us": round(t_e, 2),
+            "recall_of_exact_memory_frames": round(recall, 4)}
+
+
 def run_ours(a):
     import numpy as np
     import torch
@@ -626,10 +716,12 @@ def run_ours(a):
             "pooled keys of past frames kept from a first full pooling; each call re-pools the "
             "current chunk's frames and the queries (lf_pool_range)"))
         line["configs"] = config_report(L, lf_synth, peaks, a.config_steps, flush)
-        try:
-            line["configs"]["layer480p_1d"] = one_dim_report(L, lf_synth, peaks, a.config_steps, flush)
-        except Exception as e:  # an extra report never costs the main line
-            line["configs"]["layer480p_1d"] = {"error": repr(e)[:200]}
+        for key, fn in (("layer480p_1d", one_dim_report), ("layer480p_fp8", fp8_report),
+                        ("longvideo480p_ivf", ivf_report)):
+            try:
+                line["configs"][key] = fn(L, lf_synth, peaks, a.config_steps, flush)
+            except Exception as e:  # an extra report never costs the main line
+                line["configs"][key] = {"error": repr(e)[:200]}
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         r = _oracle_sample(w, a.cpu_budget_s, q_h, k_h, v_h)
         line["cpu_baseline"] = {"value": r["flops"] / r["t_call"] / 1e12, "unit": "TFLOP/s",
