@@ -350,10 +350,10 @@ lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, in
         return LF_ERR_ALIGN;
     const int keep = (chunk_index == 1 || topk_blocks > d.Nkv) ? d.Nkv : topk_blocks;
     if (list_cap < keep) return LF_ERR_CAP;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_NO_DEVICE;
+    int* err = nullptr;
+    if ((st = error_word(&err)) != LF_OK) return st;
     lf::SelectBlocks1dArgs a{q_pool, k_pool, block_list, block_count, d.B * d.H, d.D, d.Rq, d.Nkv,
-                             keep, list_cap, chunk_index};
+                             keep, list_cap, chunk_index, err};
     return launch_status(lf::launch_select_blocks_1d(a, static_cast<cudaStream_t>(stream)));
 }
 

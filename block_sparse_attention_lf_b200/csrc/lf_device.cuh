@@ -158,6 +158,20 @@ __device__ __forceinline__ void tma_load_4d_elect(void* smem_dst, const CUtensor
         : "memory");
 }
 
+// 1-D bulk copy (TMA, no tensor map) of `bytes` from global memory to shared memory,
+// completing on `bar`; one elected lane of a converged warp issues it. Both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load_elect(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar)
 {
     asm volatile(

@@ -46,6 +46,7 @@ struct SelectBlocks1dArgs {
     int* block_list;
     int* block_count;
     int BH, D, Rq, Nkv, kb, list_cap, chunk_index;
+    int* err;  // device error word (bounded waits of the bulk-copy ring)
 };
 
 constexpr int SEL1D_MAX_NKV = 16384;  // candidate scores held in shared memory (64 KB per scored row)

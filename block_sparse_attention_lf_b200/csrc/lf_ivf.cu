@@ -16,8 +16,9 @@
 //     clusters' frames (ties to the lower frame), plus the sink, recent and
 //     current-chunk frames, ascending. Probing every cluster is the exact selection.
 //
-// Build: one CTA per (batch, head). The k-means runs in fp64 on the fp32 frame means
-// with the oracle's operation order (distances summed over head_dim in order, member
+// Build: one CTA per (batch, head), a group of lanes per frame for the assignment and a
+// thread per (cluster, column) for the update. The k-means runs in fp64 on the fp32 frame
+// means with the oracle's operation order (distances summed over head_dim in order, member
 // sums in frame order, IEEE divisions, no fused multiply-adds), so given the same frame
 // means its labels and centroids are the oracle's, bit for bit. The result is written
 // as fp32 centroids, labels and a CSR member list grouped by cluster.
@@ -31,79 +32,109 @@
 namespace lf {
 namespace {
 
-constexpr int IDX_THREADS = 256;
+constexpr int IDX_THREADS = 512;
+constexpr int IDX_WARPS = IDX_THREADS / 32;
+constexpr size_t IDX_STAGE_MAX_SMEM = 200u * 1024u;  // frame means staged as fp64 up to this
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
 
 // ---- index build ---------------------------------------------------------------
-template <int D>
+// XS: the memory-frame means are widened to fp64 once into shared memory (when they fit);
+// otherwise every use reads and widens the fp32 value. The values are the same either way.
+template <int D, bool XS>
 __global__ void __launch_bounds__(IDX_THREADS) frame_index_kernel(const FrameIndexArgs a)
 {
+    // rows of D + 1 doubles: the lanes of a frame group read different clusters' rows at the
+    // same column, which a stride of D doubles would put in one shared-memory bank
+    constexpr int DP = D + 1;
     extern __shared__ double dsm[];
-    double* cent = dsm;                          // [C][D]
-    double* sum = cent + a.C * D;                // [C][D]
-    int* lab = reinterpret_cast<int*>(sum + a.C * D);  // [n_mem]
-    int* cnt = lab + a.n_mem;                    // [C]
-    int* off = cnt + a.C;                        // [C + 1]
-    const int tid = threadIdx.x;
+    double* cent = dsm;                                      // [C][DP]
+    double* xs = cent + a.C * DP;                            // [n_mem][DP] when XS
+    int* lab = reinterpret_cast<int*>(xs + (XS ? a.n_mem * DP : 0));  // [n_mem]
+    int* cnt = lab + a.n_mem;                           // [C]
+    int* off = cnt + a.C;                               // [C + 1]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
     const int n = a.n_mem, C = a.C;
     const float* km = a.k_frame + (static_cast<long long>(bh) * a.NF + a.n_sink) * D;
 
     for (int i = tid; i < C * D; i += IDX_THREADS) {
         const int j = i / D, d = i - j * D;
-        cent[i] = static_cast<double>(km[static_cast<long long>(j) * n / C * D + d]);
+        cent[j * DP + d] = static_cast<double>(km[static_cast<long long>(j) * n / C * D + d]);
     }
     for (int m = tid; m < n; m += IDX_THREADS) lab[m] = -1;
+    if constexpr (XS)
+        for (int i = tid; i < n * D; i += IDX_THREADS) xs[(i / D) * DP + i % D] = static_cast<double>(km[i]);
     __syncthreads();
+    // Assignment: a group of G lanes (a power of two, G >= C up to 32) per frame; lane g of
+    // the group takes clusters g, g + G, ... in order, keeping the first minimum, and the
+    // group's arg-min prefers the smaller distance, then the lower cluster: together the
+    // first minimum over the clusters in order. Each distance is summed over head_dim in
+    // order, as the oracle sums it.
+    const int G = C <= 1 ? 1 : C <= 2 ? 2 : C <= 4 ? 4 : C <= 8 ? 8 : C <= 16 ? 16 : 32;
+    const int gpw = 32 / G;  // frames per warp and round
+    const int gl = lane % G, gi = lane / G;
     for (int it = 0; it <= a.iters; ++it) {
         int changed = 0;
-        for (int m = tid; m < n; m += IDX_THREADS) {
-            const float* x = km + static_cast<long long>(m) * D;
-            int best = 0;
+        for (int m0 = warp * gpw; m0 < n; m0 += IDX_WARPS * gpw) {
+            const int m = m0 + gi;
             double bd = 0.0;
-            for (int j = 0; j < C; ++j) {
-                const double* c = cent + j * D;
-                double d2 = 0.0;
+            int best = -1;
+            if (m < n) {
+                const float* x = km + static_cast<long long>(m) * D;
+                for (int j = gl; j < C; j += G) {
+                    const double* c = cent + j * DP;
+                    double d2 = 0.0;
 #pragma unroll 8
-                for (int d = 0; d < D; ++d) {
-                    const double t = __dsub_rn(static_cast<double>(x[d]), c[d]);
-                    d2 = __dadd_rn(d2, __dmul_rn(t, t));
-                }
-                if (j == 0 || d2 < bd) {
-                    bd = d2;
-                    best = j;
+                    for (int d = 0; d < D; ++d) {
+                        const double xv = XS ? xs[m * DP + d] : static_cast<double>(__ldg(x + d));
+                        const double t = __dsub_rn(xv, c[d]);
+                        d2 = __dadd_rn(d2, __dmul_rn(t, t));
+                    }
+                    if (best < 0 || d2 < bd) {
+                        bd = d2;
+                        best = j;
+                    }
                 }
             }
-            if (lab[m] != best) {
+            for (int o = 1; o < G; o <<= 1) {  // lanes l and l ^ o are in the same group
+                const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+                const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+                if (ob >= 0 && (best < 0 || od < bd || (od == bd && ob < best))) {
+                    bd = od;
+                    best = ob;
+                }
+            }
+            if (m < n && gl == 0 && lab[m] != best) {
                 lab[m] = best;
                 changed = 1;
             }
         }
         if (!__syncthreads_or(changed) || it == a.iters) break;  // converged, or the last assignment
-        // member sums in frame order: thread d owns column d of every cluster
-        for (int i = tid; i < C * D; i += IDX_THREADS) sum[i] = 0.0;
-        if (tid < C) cnt[tid] = 0;
-        __syncthreads();
-        if (tid < D) {
-            for (int m = 0; m < n; ++m) {
-                const int j = lab[m];
-                sum[j * D + tid] = __dadd_rn(sum[j * D + tid], static_cast<double>(km[static_cast<long long>(m) * D + tid]));
-            }
-        }
-        if (tid == IDX_THREADS - 1) {  // outside the column loop (D <= 128 < IDX_THREADS)
-            for (int m = 0; m < n; ++m) cnt[lab[m]] += 1;
+        // member counts: warp w counts clusters w, w + IDX_WARPS, ...
+        for (int j = warp; j < C; j += IDX_WARPS) {
+            int c = 0;
+            for (int base = 0; base < n; base += 32)
+                c += __popc(__ballot_sync(0xffffffffu, base + lane < n && lab[base + lane] == j));
+            if (lane == 0) cnt[j] = c;
         }
         __syncthreads();
+        // centroid update: thread (j, d) sums column d of cluster j's members in frame order
+        // (the assignment above was the last reader of cent this round)
         for (int i = tid; i < C * D; i += IDX_THREADS) {
-            const int j = i / D;
-            if (cnt[j] > 0) cent[i] = __ddiv_rn(sum[i], static_cast<double>(cnt[j]));
+            const int j = i / D, d = i - j * D;
+            if (cnt[j] == 0) continue;  // an empty cluster keeps its centroid
+            double sum = 0.0;
+            for (int m = 0; m < n; ++m)
+                if (lab[m] == j)
+                    sum = __dadd_rn(sum, XS ? xs[m * DP + d] : static_cast<double>(__ldg(km + static_cast<long long>(m) * D + d)));
+            cent[j * DP + d] = __ddiv_rn(sum, static_cast<double>(cnt[j]));
         }
         __syncthreads();
     }
     // outputs: fp32 centroids, labels, and the members grouped by cluster (ascending inside)
     float* co = a.centroids + static_cast<long long>(bh) * a.C_stride * D;
-    for (int i = tid; i < C * D; i += IDX_THREADS) co[i] = static_cast<float>(cent[i]);
+    for (int i = tid; i < C * D; i += IDX_THREADS) co[i] = static_cast<float>(cent[(i / D) * DP + i % D]);
     int* lo = a.labels + static_cast<long long>(bh) * a.m_stride;
     for (int m = tid; m < n; m += IDX_THREADS) lo[m] = lab[m];
     if (tid < C) cnt[tid] = 0;
@@ -116,11 +147,10 @@ __global__ void __launch_bounds__(IDX_THREADS) frame_index_kernel(const FrameInd
     __syncthreads();
     int* oo = a.offsets + static_cast<long long>(bh) * (a.C_stride + 1);
     for (int j = tid; j <= C; j += IDX_THREADS) oo[j] = off[j];
-    // warp w compacts clusters w, w + 8, ...: ballot over the frames in order
+    // warp w compacts clusters w, w + IDX_WARPS, ...: ballot over the frames in order
     int* mo = a.members + static_cast<long long>(bh) * a.m_stride;
-    const int warp = tid >> 5, lane = tid & 31;
     const uint32_t lt = (1u << lane) - 1u;
-    for (int j = warp; j < C; j += IDX_THREADS / 32) {
+    for (int j = warp; j < C; j += IDX_WARPS) {
         int pos = off[j];
         for (int base = 0; base < n; base += 32) {
             const int m = base + lane;
@@ -296,29 +326,37 @@ cudaError_t launch_ivf_select_d(const SelectFramesIvfArgs& a, unsigned grid, cud
     return launch_ivf_select_k<D, 32>(a, grid, s);
 }
 
-template <int D>
-cudaError_t launch_index_d(const FrameIndexArgs& a, cudaStream_t s)
+template <int D, bool XS>
+cudaError_t launch_index_dx(const FrameIndexArgs& a, size_t smem, size_t smem_max, cudaStream_t s)
 {
-    const size_t smem = frame_index_smem_bytes(a.C, a.n_mem, D);
     static int configured_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(frame_index_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(frame_index_smem_bytes(IVF_MAX_CLUSTERS, IVF_MAX_MEM, D)));
+        e = cudaFuncSetAttribute(frame_index_kernel<D, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_max));
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    frame_index_kernel<D><<<static_cast<unsigned>(a.BH), IDX_THREADS, smem, s>>>(a);
+    frame_index_kernel<D, XS><<<static_cast<unsigned>(a.BH), IDX_THREADS, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_index_d(const FrameIndexArgs& a, cudaStream_t s)
+{
+    const size_t base = frame_index_smem_bytes(a.C, a.n_mem, D);
+    const size_t staged = base + static_cast<size_t>(a.n_mem) * (D + 1) * sizeof(double);
+    if (staged <= IDX_STAGE_MAX_SMEM) return launch_index_dx<D, true>(a, staged, IDX_STAGE_MAX_SMEM, s);
+    return launch_index_dx<D, false>(a, base, frame_index_smem_bytes(IVF_MAX_CLUSTERS, IVF_MAX_MEM, D), s);
 }
 
 }  // namespace
 
 size_t frame_index_smem_bytes(int C, int n_mem, int D)
 {
-    return static_cast<size_t>(2) * C * D * sizeof(double) + static_cast<size_t>(n_mem + 2 * C + 1) * sizeof(int);
+    return static_cast<size_t>(C) * (D + 1) * sizeof(double) + static_cast<size_t>(n_mem + 2 * C + 1) * sizeof(int);
 }
 
 cudaError_t launch_frame_index(const FrameIndexArgs& a, cudaStream_t s)

@@ -26,17 +26,6 @@ constexpr int POOL_THREADS = 32 * (POOL_CONSUMERS + 1);  // + one producer warp
 constexpr int POOL_SLOTS = 8;                            // ring slots of one block each
 constexpr int BLOCK_TOKENS = 64;
 
-__device__ __forceinline__ void bulk_load_elect(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar)
-{
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
-            smem_u32(smem_dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 struct PoolUnit {
     const uint16_t* src;  // first token of the frame
     float* dst;           // its block means

@@ -24,21 +24,23 @@ __device__ __forceinline__ void transpose_reduce_sum(float (&v)[32], int lane)
     }
 }
 
-template <int EPL>
+// SHARED: p points into shared memory (plain load); otherwise read-only global memory.
+template <int EPL, bool SHARED = false>
 __device__ __forceinline__ void load_lane(float (&dst)[EPL], const float* p)
 {
     if constexpr (EPL == 4) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(p));
+        const float4 t = SHARED ? *reinterpret_cast<const float4*>(p) : __ldg(reinterpret_cast<const float4*>(p));
         dst[0] = t.x; dst[1] = t.y; dst[2] = t.z; dst[3] = t.w;
     } else {
-        const float2 t = __ldg(reinterpret_cast<const float2*>(p));
+        const float2 t = SHARED ? *reinterpret_cast<const float2*>(p) : __ldg(reinterpret_cast<const float2*>(p));
         dst[0] = t.x; dst[1] = t.y;
     }
 }
 
 // Scores of candidates base..base+31 (rows of `rows`, D floats each, only the
-// first n are real); returns the score of candidate base+lane (0 if beyond n).
-template <int D>
+// first n are real; in shared memory when SHARED); returns the score of candidate
+// base+lane (0 if beyond n).
+template <int D, bool SHARED = false>
 __device__ __forceinline__ float score_group(const float (&qv)[D / 32], const float* rows, int base,
                                              int n, int lane)
 {
@@ -49,7 +51,7 @@ __device__ __forceinline__ float score_group(const float (&qv)[D / 32], const fl
         part[c] = 0.f;
         if (base + c < n) {
             float kv[EPL];
-            load_lane<EPL>(kv, rows + static_cast<long long>(base + c) * D + lane * EPL);
+            load_lane<EPL, SHARED>(kv, rows + static_cast<long long>(base + c) * D + lane * EPL);
 #pragma unroll
             for (int e = 0; e < EPL; ++e) part[c] = fmaf(qv[e], kv[e], part[c]);
         }

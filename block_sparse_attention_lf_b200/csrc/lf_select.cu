@@ -194,17 +194,37 @@ __global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(
 
 // One-dimensional selection (the single-granularity variant of the ablation in
 // "南洋理工大学打造视频生成新引擎", 163.com, section 4): every KV block of the head is a
-// candidate. One CTA per scored row: its warps score groups of 32 candidates into 32-bit
-// orderable scores in shared memory; then one warp finds the exact score T of the kb-th
-// largest bit by bit from the top (32 rounds of warp ballot counts, no block barrier) and
-// writes, in index order, every candidate scoring above T and the lowest-indexed ones
-// scoring exactly T until kb are kept: the order of the two-level kernels' 64-bit keys
-// (score, then lower index), so the lists are those of a full sort.
+// candidate. One CTA per scored row. A producer warp streams the head's pooled keys in
+// groups of 32 candidates (16 KB at head_dim 128) into a 4-slot shared-memory ring with
+// 1-D bulk copies; consumer warp w owns slot w and scores groups w, w + 4, ... into
+// 32-bit orderable scores in shared memory, so each slot's uses are waited for in order
+// by one warp. The four consumer warps then find the exact score T of the kb-th largest
+// bit by bit from the top (32 rounds: per-thread counts, one warp reduction, the four
+// warp counts through shared memory, one barrier per round) and write, in index order,
+// every candidate scoring above T and the lowest-indexed ones scoring exactly T until kb
+// are kept: the order of the two-level kernels' 64-bit keys (score, then lower index),
+// so the list is that of a full sort.
+constexpr int SEL1D_CONSUMERS = 4;
+constexpr int SEL1D_THREADS = 32 * (SEL1D_CONSUMERS + 1);
+constexpr int SEL1D_CT = 32 * SEL1D_CONSUMERS;  // consumer threads
+
 template <int D>
-__global__ void __launch_bounds__(SEL_THREADS) select_blocks_1d_kernel(const SelectBlocks1dArgs a)
+constexpr size_t sel1d_ring_bytes()
+{
+    return static_cast<size_t>(SEL1D_CONSUMERS) * 32u * D * sizeof(float);
+}
+
+template <int D>
+__global__ void __launch_bounds__(SEL1D_THREADS) select_blocks_1d_kernel(const SelectBlocks1dArgs a)
 {
     constexpr int EPL = D / 32;
-    extern __shared__ uint32_t sc[];  // [Nkv] orderable scores
+    constexpr int GROUP_FLOATS = 32 * D;
+    extern __shared__ __align__(128) uint8_t sm1d[];
+    float* ring = reinterpret_cast<float*>(sm1d);                                // [SEL1D_CONSUMERS][32][D]
+    uint32_t* sc = reinterpret_cast<uint32_t*>(sm1d + sel1d_ring_bytes<D>());    // [Nkv]
+    __shared__ uint64_t full[SEL1D_CONSUMERS], empty[SEL1D_CONSUMERS];
+    __shared__ int wc[2][2][SEL1D_CONSUMERS];  // per-warp counts, double-buffered by round parity
+    __shared__ int abort_word;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long row = blockIdx.x;
     const int n = a.Nkv;
@@ -213,66 +233,128 @@ __global__ void __launch_bounds__(SEL_THREADS) select_blocks_1d_kernel(const Sel
     const int keep = (a.chunk_index == 1 || a.kb >= n) ? n : a.kb;
     if (threadIdx.x == 0) a.block_count[row] = keep;
     if (keep == n) {
-        for (int g = threadIdx.x; g < n; g += SEL_THREADS) out[g] = g;
+        for (int g = threadIdx.x; g < n; g += SEL1D_THREADS) out[g] = g;
         return;
     }
-    float qv[EPL];
-    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
-    const float* kblk = a.k_pool + static_cast<long long>(bh) * n * D;
-    for (int grp = warp; grp * 32 < n; grp += SEL_WARPS) {
-        const float s = score_group<D>(qv, kblk, grp * 32, n, lane);
-        if (grp * 32 + lane < n) sc[grp * 32 + lane] = orderable(s);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SEL1D_CONSUMERS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        abort_word = 0;
+        fence_mbar_init();
     }
     __syncthreads();
-    if (warp != 0) return;
-    // T = the largest 32-bit value with at least `keep` scores >= T, built bit by bit
+    volatile int* abort_flag = &abort_word;
+    const float* kblk = a.k_pool + static_cast<long long>(bh) * n * D;
+    const int n_groups = (n + 31) / 32;
+    if (warp == SEL1D_CONSUMERS) {
+        // ---------------------------------------------------------------- producer
+        int g = 0;
+        for (; g < n_groups; ++g) {
+            const int s = g % SEL1D_CONSUMERS;
+            if (!mbar_wait(&empty[s], static_cast<uint32_t>(((g / SEL1D_CONSUMERS) & 1) ^ 1), abort_flag, a.err, 0x50))
+                break;
+            const uint32_t bytes = static_cast<uint32_t>(min(32, n - 32 * g)) * D * sizeof(float);
+            mbar_arrive_expect_tx_elect(&full[s], bytes);
+            bulk_load_elect(ring + s * GROUP_FLOATS, kblk + static_cast<long long>(g) * GROUP_FLOATS, bytes, &full[s]);
+        }
+        if (g < n_groups)  // aborted: let the copies already issued land before the CTA exits
+            for (int g2 = max(0, g - SEL1D_CONSUMERS); g2 < g; ++g2)
+                mbar_drain(&full[g2 % SEL1D_CONSUMERS], static_cast<uint32_t>((g2 / SEL1D_CONSUMERS) & 1), 10000000ull);
+        return;
+    }
+    // -------------------------------------------------------------------- consumers
+    float qv[EPL];
+    load_lane<EPL>(qv, a.q_pool + row * D + lane * EPL);
+    for (int g = warp; g < n_groups; g += SEL1D_CONSUMERS) {
+        if (!mbar_wait(&full[warp], static_cast<uint32_t>((g / SEL1D_CONSUMERS) & 1), abort_flag, a.err, 0x51)) break;
+        const int cnt = min(32, n - 32 * g);
+        const float s = score_group<D, true>(qv, ring + warp * GROUP_FLOATS, 0, cnt, lane);
+        if (lane < cnt) sc[32 * g + lane] = orderable(s);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[warp]);
+    }
+    // scores complete (or the CTA gave up: the same decision in every consumer thread)
+    if (named_bar_or(1, SEL1D_CT, *abort_flag != 0)) return;
+    const int tid = threadIdx.x;
+    // T = the largest 32-bit value with at least `keep` scores >= T, built bit by bit.
+    // Round `bit` writes wc[bit & 1][0]; a buffer is rewritten two rounds later, after
+    // every consumer thread has passed the barrier of the round in between.
     uint32_t prefix = 0;
     for (int bit = 31; bit >= 0; --bit) {
         const uint32_t cand = prefix | (1u << bit);
         int c = 0;
-        for (int base = 0; base < n; base += 32) {
-            const int g = base + lane;
-            c += __popc(__ballot_sync(0xffffffffu, g < n && sc[g] >= cand));
-        }
-        if (c >= keep) prefix = cand;
+        for (int g = tid; g < n; g += SEL1D_CT) c += sc[g] >= cand ? 1 : 0;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) wc[bit & 1][0][warp] = c;
+        named_bar_sync(1, SEL1D_CT);
+        int tot = 0;
+#pragma unroll
+        for (int w = 0; w < SEL1D_CONSUMERS; ++w) tot += wc[bit & 1][0][w];
+        if (tot >= keep) prefix = cand;
     }
     int above = 0;
-    for (int base = 0; base < n; base += 32) {
-        const int g = base + lane;
-        above += __popc(__ballot_sync(0xffffffffu, g < n && sc[g] > prefix));
+    {
+        int c = 0;
+        for (int g = tid; g < n; g += SEL1D_CT) c += sc[g] > prefix ? 1 : 0;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) wc[1][1][warp] = c;  // not used by the rounds above
+        named_bar_sync(1, SEL1D_CT);
+#pragma unroll
+        for (int w = 0; w < SEL1D_CONSUMERS; ++w) above += wc[1][1][w];
     }
     const int need = keep - above;  // scores equal to T still to take, lowest index first
-    int pos = 0, eq_seen = 0;
+    // Index-order compaction, SEL1D_CT candidates per chunk. Before candidate g: gt_before
+    // scores above T and eq_before equal to T; g goes to gt_before + min(eq_before, need).
     const uint32_t lt = (1u << lane) - 1u;
-    for (int base = 0; base < n; base += 32) {
-        const int g = base + lane;
+    int gt_base = 0, eq_base = 0;
+    for (int c0 = 0, it = 0; c0 < n; c0 += SEL1D_CT, ++it) {
+        const int g = c0 + tid;
         const uint32_t v = g < n ? sc[g] : 0u;
+        const bool gt = g < n && v > prefix;
         const bool eq = g < n && v == prefix;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-        const bool take = (g < n && v > prefix) || (eq && eq_seen + __popc(eqm & lt) < need);
-        const uint32_t tm = __ballot_sync(0xffffffffu, take);
-        if (take) out[pos + __popc(tm & lt)] = g;
-        pos += __popc(tm);
-        eq_seen += __popc(eqm);
+        const uint32_t gm = __ballot_sync(0xffffffffu, gt);
+        const uint32_t em = __ballot_sync(0xffffffffu, eq);
+        const int b = it & 1;
+        if (lane == 0) {
+            wc[b][0][warp] = __popc(gm);
+            wc[b][1][warp] = __popc(em);
+        }
+        named_bar_sync(1, SEL1D_CT);
+        int pg = 0, pe = 0, tg = 0, te = 0;
+#pragma unroll
+        for (int w = 0; w < SEL1D_CONSUMERS; ++w) {
+            const int x = wc[b][0][w], y = wc[b][1][w];
+            pg += w < warp ? x : 0;
+            pe += w < warp ? y : 0;
+            tg += x;
+            te += y;
+        }
+        const int gt_before = gt_base + pg + __popc(gm & lt);
+        const int eq_before = eq_base + pe + __popc(em & lt);
+        if (gt || (eq && eq_before < need)) out[gt_before + min(eq_before, need)] = g;
+        gt_base += tg;
+        eq_base += te;
     }
 }
 
 template <int D>
 cudaError_t launch_blocks_1d_d(const SelectBlocks1dArgs& a, cudaStream_t s)
 {
-    const size_t smem = static_cast<size_t>(a.Nkv) * sizeof(uint32_t);
+    const size_t smem = sel1d_ring_bytes<D>() + static_cast<size_t>(a.Nkv) * sizeof(uint32_t);
     static int configured_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
         e = cudaFuncSetAttribute(select_blocks_1d_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(SEL1D_MAX_NKV * sizeof(uint32_t)));
+                                 static_cast<int>(sel1d_ring_bytes<D>() + SEL1D_MAX_NKV * sizeof(uint32_t)));
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(a.BH) * a.Rq);
-    select_blocks_1d_kernel<D><<<grid, SEL_THREADS, smem, s>>>(a);
+    select_blocks_1d_kernel<D><<<grid, SEL1D_THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }
 

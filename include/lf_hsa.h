@@ -224,7 +224,10 @@ LF_API lf_status lf_select_mask(const lf_hsa_shape* shape, int32_t chunk_index, 
  * Among equal scores the lower block index wins. Nkv is limited to 16384.
  * Errors: LF_ERR_NULL, LF_ERR_ALIGN, LF_ERR_SHAPE (also Nkv > 16384),
  * LF_ERR_TOPK, LF_ERR_CAP (list_cap below the kept count), LF_ERR_ARG
- * (chunk_index < 1), LF_ERR_NO_DEVICE, LF_ERR_CUDA.
+ * (chunk_index < 1), LF_ERR_NO_DEVICE, LF_ERR_CUDA. The kernel streams k_pool
+ * through shared memory with bulk copies whose waits are bounded (1 s); a wait
+ * that expires sets the device error word (lf_get_device_error) and the row's
+ * list is left unwritten.
  */
 LF_API lf_status lf_select_blocks_1d(const lf_hsa_shape* shape, int32_t chunk_index, int32_t topk_blocks,
                               const float* q_pool, const float* k_pool, int32_t* block_list,

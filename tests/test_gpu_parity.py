@@ -242,8 +242,17 @@ def test_split_matches_unsplit_layer480p():
     assert d <= parity.OUT_MAX_ABS, d
 
 
+# Shapes for the selection launch only: many memory frames (200 and 805 memory frames of
+# 8 blocks; 7 and 26 frame-key slots per lane in the frame level).
+LARGE_SELECTION = [
+    ("200_memory_frames", 1, 1, 64, 512, (1, 200, 1, 3), 2, 8, 3, 1.0, 0),
+    ("805_memory_frames", 1, 1, 64, 512, (1, 805, 1, 3), 2, 8, 3, 1.0, 0),
+]
+
+
 @pytest.mark.parametrize("name,chunk", [("ragged_d128", 2), ("ragged_d64_odd_lists", 2), ("dense_first_chunk", 1),
-                                        ("no_memory_frames", 2), ("layer480p", 2), ("longvideo480p", 2)])
+                                        ("no_memory_frames", 2), ("layer480p", 2), ("longvideo480p", 2),
+                                        ("200_memory_frames", 2), ("805_memory_frames", 2)])
 def test_fused_selection_equals_two_kernels(name, chunk):
     """lf_select_mask (both levels in one launch) writes exactly what lf_select_frames followed by
     lf_select_blocks write: same frame rows, lists and counts, bit for bit."""
@@ -256,7 +265,7 @@ def test_fused_selection_equals_two_kernels(name, chunk):
         n_sel = L.lf_frames_selected(ls, chunk, kf)
         kb = w.topk_blocks or L.lf_blocks_for_sparsity(w.sparsity, ls.Nkv, n_sel, ls.bpf)
     else:
-        case = next(c for c in SMALL if c[0] == name)
+        case = next(c for c in SMALL + LARGE_SELECTION if c[0] == name)
         _, B, H, D, F, (ns, nm, nr, nc), _, kf, kb, kscale, _ = case
         ls = L.LfShape.make(B, H, D, F, ns + nm + nr + nc, ns, nr, nc)
         q, k, v = _rand(zlib.crc32(name.encode()) % 1000, B, H, nc * F, ls.n_frames * F, D, kscale)

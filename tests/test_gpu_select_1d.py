@@ -73,6 +73,9 @@ CASES = [
     ("dense_first_chunk", 1, 2, 128, 260, (0, 0, 0, 3), 1, 4),
     ("keep_everything", 1, 2, 128, 190, (1, 2, 1, 2), 2, 10 ** 6),
     ("525_candidates", 1, 1, 128, 1560, (1, 16, 1, 3), 2, 108),
+    # many candidates per row (1,600 and 6,480 KV blocks of 8 per frame)
+    ("1600_candidates", 1, 1, 64, 512, (1, 195, 1, 3), 2, 40),
+    ("6480_candidates", 1, 1, 64, 512, (1, 805, 1, 3), 2, 50),
 ]
 
 
