@@ -51,6 +51,9 @@ def _args():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the per-config report (all five workloads, rollout per chunk)")
     p.add_argument("--config-steps", type=int, default=30)
+    p.add_argument("--only-report", choices=["layer480p_1d", "layer480p_fp8", "longvideo480p_ivf"], default=None,
+                   help="run only this extra report after the main line (skips the other configs); "
+                        "used to profile one of its kernels")
     p.add_argument("--strong", action="store_true",
                    help="N > 1: split one call's (batch, head) units across the ranks (strong scaling); "
                         "default: each rank takes a whole workload's units of a call whose batch grows "
@@ -710,14 +713,19 @@ def run_ours(a):
         "clocks": clk.summary(),
         "wall_s_timed_region": wall,
     }
-    if rank == 0 and not a.no_configs:
+    extra = (("layer480p_1d", one_dim_report), ("layer480p_fp8", fp8_report), ("longvideo480p_ivf", ivf_report))
+    if rank == 0 and a.only_report:
+        line["configs"] = {}
+        for key, fn in extra:
+            if key == a.only_report:
+                line["configs"][key] = fn(L, lf_synth, peaks, a.config_steps, flush)
+    elif rank == 0 and not a.no_configs:
         mc = measure_call(L, shape, w.chunk_index, w.topk_frames, kb, q, k, v, a.config_steps, 3, flush, cached=True)
         line["cached_pooled_keys"] = dict(_summary(mc, peaks), note=(
             "pooled keys of past frames kept from a first full pooling; each call re-pools the "
             "current chunk's frames and the queries (lf_pool_range)"))
         line["configs"] = config_report(L, lf_synth, peaks, a.config_steps, flush)
-        for key, fn in (("layer480p_1d", one_dim_report), ("layer480p_fp8", fp8_report),
-                        ("longvideo480p_ivf", ivf_report)):
+        for key, fn in extra:
             try:
                 line["configs"][key] = fn(L, lf_synth, peaks, a.config_steps, flush)
             except Exception as e:  # an extra report never costs the main line

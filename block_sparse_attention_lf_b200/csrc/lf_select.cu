@@ -108,6 +108,34 @@ __global__ void __launch_bounds__(SEL_THREADS) select_frames_kernel(const Select
     frames_of_row<D, KPL>(a, row, lane, qv, a.frame_sel + row * a.n_sel, nullptr);
 }
 
+// The top-k_b of a frame's block keys (key slot i of lane l = block i * 32 + l, 0 = none) by
+// rank counting (rank = number of larger keys), written ascending by a ballot compaction.
+template <int KPL>
+__device__ __forceinline__ void write_top_blocks(const SelectBlocksArgs& a, int* out, const uint64_t (&key)[KPL],
+                                                 int tau, int lane)
+{
+    int rank[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) rank[i] = 0;
+    for (int src = 0; src < 32; ++src) {
+#pragma unroll
+        for (int i2 = 0; i2 < KPL; ++i2) {
+            const uint64_t o = __shfl_sync(0xffffffffu, key[i2], src);
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) rank[i] += (o > key[i]) ? 1 : 0;
+        }
+    }
+    int prefix = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const bool keep = key[i] != 0ull && rank[i] < a.kb;
+        const uint32_t mask = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[prefix + __popc(mask & lt)] = tau * a.bpf + i * 32 + lane;
+        prefix += __popc(mask);
+    }
+}
+
 // The top-k_b blocks of selected frame slot s (frame tau) of scored row `row` (one
 // warp), written ascending into the row's list at s * k_b. KPL = ceil(bpf / 32).
 template <int D, int KPL>
@@ -133,27 +161,7 @@ __device__ __forceinline__ void blocks_of_frame(const SelectBlocksArgs& a, long 
         key[i] = (j < a.bpf) ? make_key(sc, j) : 0ull;
     }
 
-    int rank[KPL];
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) rank[i] = 0;
-    for (int src = 0; src < 32; ++src) {
-#pragma unroll
-        for (int i2 = 0; i2 < KPL; ++i2) {
-            const uint64_t o = __shfl_sync(0xffffffffu, key[i2], src);
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) rank[i] += (o > key[i]) ? 1 : 0;
-        }
-    }
-
-    int prefix = 0;
-    const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-        const bool keep = key[i] != 0ull && rank[i] < a.kb;
-        const uint32_t mask = __ballot_sync(0xffffffffu, keep);
-        if (keep) out[prefix + __popc(mask & lt)] = tau * a.bpf + i * 32 + lane;
-        prefix += __popc(mask);
-    }
+    write_top_blocks<KPL>(a, out, key, tau, lane);
 }
 
 // One warp per (row, selected-frame slot).
@@ -190,6 +198,207 @@ __global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(
     if (warp == 0) frames_of_row<D, KPLF>(fa, row, lane, qv, fa.frame_sel + row * fa.n_sel, sel_s);
     __syncthreads();
     for (int s = warp; s < ba.n_sel; s += n_warps) blocks_of_frame<D, KPLB>(ba, row, s, sel_s[s], lane, qv);
+}
+
+// ---- one-dimensional selection, tiled, through a bulk-copy ring ----------------------
+// One CTA per tile of TR_ROWS scored rows (query blocks) of one head. A producer warp
+// streams the head's pooled keys in groups of 32 candidates (16 KB at head_dim 128) into a
+// TR_SLOTS-slot shared-memory ring with 1-D bulk copies, so each pooled key crosses
+// L2 -> SM once per tile instead of once per row. Consumer warp w scores rows 2(w % 4) and
+// 2(w % 4) + 1 against the groups g with g % 2 == w / 4: each candidate slice read from
+// shared memory feeds two inner products. Groups are laid out as in the one-row kernel
+// (32 consecutive blocks from the head's first), so every score, and with it every list,
+// is bit-identical to its. Slot s only ever holds groups of parity s % 2 and is consumed by
+// the same four warps, in order. (The two-level selection tiled the same way, all of a
+// head's blocks scored per tile, ran at 34.8 us against 23.6 us for select_fused_kernel,
+// which scores only the selected frames' blocks; it was not kept.)
+constexpr int TR_ROWS = 8;
+constexpr int TR_CONSUMERS = 8;
+constexpr int TR_CT = 32 * TR_CONSUMERS;  // consumer threads
+constexpr int TR_THREADS = TR_CT + 32;    // + the producer warp
+constexpr int TR_SLOTS = 4;               // even: slot s holds groups of parity s % 2
+constexpr int TR_1D_MAX_NKV = 2048;       // scores of a row in registers (64 per lane); beyond: the one-row kernel
+
+template <int D>
+constexpr size_t tr_ring_bytes()
+{
+    return static_cast<size_t>(TR_SLOTS) * 32u * D * sizeof(float);
+}
+
+struct TileRing {
+    uint64_t full[TR_SLOTS], empty[TR_SLOTS];
+    int abort;
+};
+
+// Groups of 32 consecutive candidates of the head (the last one may be shorter).
+struct TileGroups {
+    int n, n_groups;
+    __device__ __forceinline__ explicit TileGroups(int n_) : n(n_), n_groups((n_ + 31) / 32) {}
+    __device__ __forceinline__ int base(int g) const { return 32 * g; }
+    __device__ __forceinline__ int count(int g) const { return min(32, n - 32 * g); }
+};
+
+// The two-row scoring of score_group (SHARED: rows in shared memory).
+template <int D, bool SHARED>
+__device__ __forceinline__ void score_group2(const float (&q0)[D / 32], const float (&q1)[D / 32], const float* rows,
+                                             int n, int lane, float& s0, float& s1)
+{
+    constexpr int EPL = D / 32;
+    float p0[32], p1[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        p0[c] = 0.f;
+        p1[c] = 0.f;
+        if (c < n) {
+            float kv[EPL];
+            load_lane<EPL, SHARED>(kv, rows + static_cast<long long>(c) * D + lane * EPL);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                p0[c] = fmaf(q0[e], kv[e], p0[c]);
+                p1[c] = fmaf(q1[e], kv[e], p1[c]);
+            }
+        }
+    }
+    transpose_reduce_sum(p0, lane);
+    transpose_reduce_sum(p1, lane);
+    s0 = p0[0];
+    s1 = p1[0];
+}
+
+__device__ __forceinline__ void tile_ring_init(TileRing& r)
+{
+    for (int s = 0; s < TR_SLOTS; ++s) {
+        mbar_init(&r.full[s], 1);
+        mbar_init(&r.empty[s], TR_CONSUMERS / 2);  // the four warps of the slot's parity
+    }
+    r.abort = 0;
+    fence_mbar_init();
+}
+
+// Producer warp: every group of the head, in order.
+template <int D>
+__device__ __forceinline__ void tile_produce(TileRing& r, const TileGroups& tg, const float* kblk, float* ring, int* err)
+{
+    volatile int* abort_flag = &r.abort;
+    int g = 0;
+    for (; g < tg.n_groups; ++g) {
+        const int s = g % TR_SLOTS;
+        if (!mbar_wait(&r.empty[s], static_cast<uint32_t>(((g / TR_SLOTS) & 1) ^ 1), abort_flag, err, 0x52)) break;
+        const uint32_t bytes = static_cast<uint32_t>(tg.count(g)) * D * sizeof(float);
+        mbar_arrive_expect_tx_elect(&r.full[s], bytes);
+        bulk_load_elect(ring + s * 32 * D, kblk + static_cast<long long>(tg.base(g)) * D, bytes, &r.full[s]);
+    }
+    if (g < tg.n_groups)  // aborted: let the copies already issued land before the CTA exits
+        for (int g2 = max(0, g - TR_SLOTS); g2 < g; ++g2)
+            mbar_drain(&r.full[g2 % TR_SLOTS], static_cast<uint32_t>((g2 / TR_SLOTS) & 1), 10000000ull);
+}
+
+// Consumer warps: the tile's scores into sc[TR_ROWS][n]; rows past rows_valid score with a
+// zero query and are never read. Returns false when the CTA gave up; the answer is the same
+// in every consumer thread, and the call is the barrier after which sc is complete.
+template <int D>
+__device__ __forceinline__ bool tile_score(TileRing& r, const TileGroups& tg, const float* q_pool, long long row0,
+                                           int rows_valid, int n, const float* ring, float* sc, int* err, int warp,
+                                           int lane)
+{
+    constexpr int EPL = D / 32;
+    volatile int* abort_flag = &r.abort;
+    const int ra = 2 * (warp & 3), rb = ra + 1, par = warp >> 2;
+    float q0[EPL], q1[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        q0[e] = 0.f;
+        q1[e] = 0.f;
+    }
+    if (ra < rows_valid) load_lane<EPL>(q0, q_pool + (row0 + ra) * D + lane * EPL);
+    if (rb < rows_valid) load_lane<EPL>(q1, q_pool + (row0 + rb) * D + lane * EPL);
+    for (int g = par; g < tg.n_groups; g += 2) {
+        const int s = g % TR_SLOTS;
+        if (!mbar_wait(&r.full[s], static_cast<uint32_t>((g / TR_SLOTS) & 1), abort_flag, err, 0x53)) break;
+        const int base = tg.base(g), cnt = tg.count(g);
+        float s0, s1;
+        score_group2<D, true>(q0, q1, ring + s * 32 * D, cnt, lane, s0, s1);
+        if (lane < cnt) {
+            sc[ra * n + base + lane] = s0;
+            sc[rb * n + base + lane] = s1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&r.empty[s]);
+    }
+    return !named_bar_or(1, TR_CT, *abort_flag != 0);
+}
+
+// One-dimensional selection over the tile's scores: each warp its row, the row's scores in
+// registers (VPL per lane, candidate 32 i + lane in slot i); the threshold score T of the
+// kept count is built bit by bit (32 rounds of per-lane counts and one warp reduction), then
+// every candidate above T and the lowest-indexed ones equal to T are written in index order.
+template <int D, int VPL>
+__global__ void __launch_bounds__(TR_THREADS) select_1d_tile_kernel(const SelectBlocks1dArgs a)
+{
+    extern __shared__ __align__(128) uint8_t tr_smem[];
+    __shared__ TileRing rc;
+    const int n = a.Nkv;
+    float* ring = reinterpret_cast<float*>(tr_smem);
+    float* sc = reinterpret_cast<float*>(tr_smem + tr_ring_bytes<D>());  // [TR_ROWS][n]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tiles = (a.Rq + TR_ROWS - 1) / TR_ROWS;
+    const int bh = static_cast<int>(blockIdx.x / tiles);
+    const int r_in = static_cast<int>(blockIdx.x - static_cast<long long>(bh) * tiles) * TR_ROWS;
+    const int rows_valid = min(TR_ROWS, a.Rq - r_in);
+    const long long row0 = static_cast<long long>(bh) * a.Rq + r_in;
+    const int keep = (a.chunk_index == 1 || a.kb >= n) ? n : a.kb;
+    if (keep == n) {
+        if (warp < rows_valid) {
+            int* out = a.block_list + (row0 + warp) * a.list_cap;
+            if (lane == 0) a.block_count[row0 + warp] = keep;
+            for (int g = lane; g < n; g += 32) out[g] = g;
+        }
+        return;
+    }
+    const TileGroups tg(n);
+    if (threadIdx.x == 0) tile_ring_init(rc);
+    __syncthreads();
+    if (warp == TR_CONSUMERS) {
+        tile_produce<D>(rc, tg, a.k_pool + static_cast<long long>(bh) * n * D, ring, a.err);
+        return;
+    }
+    if (!tile_score<D>(rc, tg, a.q_pool, row0, rows_valid, n, ring, sc, a.err, warp, lane)) return;
+    if (warp >= rows_valid) return;
+    const long long row = row0 + warp;
+    int* out = a.block_list + row * a.list_cap;
+    if (lane == 0) a.block_count[row] = keep;
+    uint32_t v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int g = 32 * i + lane;
+        v[i] = g < n ? orderable(sc[warp * n + g]) : 0u;
+    }
+    uint32_t prefix = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = prefix | (1u << bit);
+        int c = 0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) c += (32 * i + lane < n && v[i] >= cand) ? 1 : 0;
+        if (__reduce_add_sync(0xffffffffu, c) >= keep) prefix = cand;
+    }
+    int above = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) above += (32 * i + lane < n && v[i] > prefix) ? 1 : 0;
+    const int need = keep - __reduce_add_sync(0xffffffffu, above);  // scores equal to T still to take
+    int pos = 0, eq_seen = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int g = 32 * i + lane;
+        const bool valid = g < n;
+        const bool eq = valid && v[i] == prefix;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool take = (valid && v[i] > prefix) || (eq && eq_seen + __popc(eqm & lt) < need);
+        const uint32_t tm = __ballot_sync(0xffffffffu, take);
+        if (take) out[pos + __popc(tm & lt)] = g;
+        pos += __popc(tm);
+        eq_seen += __popc(eqm);
+    }
 }
 
 // One-dimensional selection (the single-granularity variant of the ablation in
@@ -339,9 +548,48 @@ __global__ void __launch_bounds__(SEL1D_THREADS) select_blocks_1d_kernel(const S
     }
 }
 
+// Shared-memory opt-in of a tiled kernel, once per device.
+template <typename Kernel>
+cudaError_t tile_smem_optin(Kernel k, int& configured_device, size_t bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    return cudaSuccess;
+}
+
+template <int D, int VPL>
+cudaError_t launch_1d_tile(const SelectBlocks1dArgs& a, cudaStream_t s)
+{
+    static int configured_device = -1;
+    cudaError_t e = tile_smem_optin(select_1d_tile_kernel<D, VPL>, configured_device,
+                                    tr_ring_bytes<D>() + TR_ROWS * TR_1D_MAX_NKV * sizeof(float));
+    if (e != cudaSuccess) return e;
+    const long long tiles = (a.Rq + TR_ROWS - 1) / TR_ROWS;
+    select_1d_tile_kernel<D, VPL><<<static_cast<unsigned>(static_cast<long long>(a.BH) * tiles), TR_THREADS,
+                                    tr_ring_bytes<D>() + static_cast<size_t>(TR_ROWS) * a.Nkv * sizeof(float), s>>>(a);
+    return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_blocks_1d_d(const SelectBlocks1dArgs& a, cudaStream_t s)
 {
+    if (a.Nkv <= TR_1D_MAX_NKV) {
+        const int vpl = (a.Nkv + 31) / 32;
+        if (vpl <= 4) return launch_1d_tile<D, 4>(a, s);
+        if (vpl <= 8) return launch_1d_tile<D, 8>(a, s);
+        if (vpl <= 16) return launch_1d_tile<D, 16>(a, s);
+        if (vpl <= 20) return launch_1d_tile<D, 20>(a, s);
+        if (vpl <= 24) return launch_1d_tile<D, 24>(a, s);
+        if (vpl <= 32) return launch_1d_tile<D, 32>(a, s);
+        if (vpl <= 48) return launch_1d_tile<D, 48>(a, s);
+        return launch_1d_tile<D, 64>(a, s);
+    }
     const size_t smem = sel1d_ring_bytes<D>() + static_cast<size_t>(a.Nkv) * sizeof(uint32_t);
     static int configured_device = -1;
     int dev = 0;
