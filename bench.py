@@ -537,7 +537,11 @@ def fp8_report(L, lf_synth, peaks, steps, flush):
     attn8 = lambda: L.lf_block_sparse_attn_fp8(shape, q8, k8, qs, ks, v, b.block_list, b.block_count, b.list_cap,
                                                0.0, out8, call.workspace, call.tail_pieces)
     for _ in range(3):
-        quant_q(); quant_k(); attn8()
+        quant_q(); quant_k()
+        # an NVTX range lets a profiler pick out the e4m3 attention launches
+        torch.cuda.nvtx.range_push("lf_fp8_attn")
+        attn8()
+        torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     st, detail = L.lf_get_device_error()
     if st != 0:

@@ -26,7 +26,10 @@
 //     MN-major (LBO = 1 KB between head-dim panels, SBO = 2 KB between 8-row
 //     groups). Frames whose token count is not a multiple of 8, and head_dim
 //     64, use 2-D boxes per 64-wide panel into a plain [panel][row] layout.
-//     K arrives per tile (ring of 2 tiles), V per block (ring of 4 blocks).
+//     The K ring holds two tiles but is filled and released per block: each block's
+//     score MMAs (M = 64, N = 64, the same rate as N = 128) release its slot, so the next
+//     step's first block loads while the tile's second block is still being scored
+//     (1-2 % faster than releasing whole tiles). V arrives per block (ring of 4 blocks).
 //   * Warp roles (384 threads): warp 0 issues the Q and K loads, warp 1 the V
 //     loads, warp 2 allocates TMEM and issues the score MMAs, warp 3 issues the
 //     PV MMAs, warps 4-11 are two softmax warpgroups. Warpgroup g takes
@@ -120,7 +123,7 @@ struct AttnAux {
     static constexpr int KSLOTS = Rings<F8>::K;
     static constexpr int VSLOTS = Rings<F8>::V;
     uint64_t q_full;
-    uint64_t k_full[KSLOTS], k_empty[KSLOTS];
+    uint64_t k_full[2 * KSLOTS], k_empty[2 * KSLOTS];  // per KV block of the K ring
     uint64_t v_full[VSLOTS], v_empty[VSLOTS];
     uint64_t s_full[SBUFS], s_free[SBUFS];
     uint64_t p_full[2], p_empty[2];  // per warpgroup: its P written / its last PV done
@@ -257,7 +260,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (tid == 0) {
         mbar_init(&x.q_full, 1);
-        for (int s = 0; s < KSLOTS; ++s) { mbar_init(&x.k_full[s], 1); mbar_init(&x.k_empty[s], 1); }
+        for (int s = 0; s < 2 * KSLOTS; ++s) { mbar_init(&x.k_full[s], 1); mbar_init(&x.k_empty[s], 1); }
         for (int s = 0; s < VSLOTS; ++s) { mbar_init(&x.v_full[s], 1); mbar_init(&x.v_empty[s], 1); }
         for (int s = 0; s < SBUFS; ++s) {
             mbar_init(&x.s_full[s], 1);
@@ -308,37 +311,32 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (int p = 0; p < L::NPQ; ++p)
                 tma_load_2d_elect(smem + L::OFF_Q + p * L::PANEL_Q, mq, p * 64, q_row0, &x.q_full);
             int armed = 0;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int nb = min(2, cnt - 2 * t);
-                int rows[2] = {0, 0}, first[2] = {0, 0};
-                for (int h = 0; h < nb; ++h) {
-                    rows[h] = block_rows(a, list_entry(x.lst, lst, 2 * t + h), bh, &first[h]);
-                    if (rows[h] == 0 && lane == 0) record_error(a.err, DEVERR_LIST | 2);
-                }
-                const uint32_t bytes = static_cast<uint32_t>((rows[0] + rows[1]) * 128 * L::NPQ);
-                const int s = t % KSLOTS;
-                if (!mbar_wait(&x.k_empty[s], ((t / KSLOTS) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
-                if (bytes) mbar_arrive_expect_tx_elect(&x.k_full[s], bytes);
-                else mbar_arrive_elect(&x.k_full[s]);
-                uint8_t* slot = smem + L::OFF_K + s * L::K_SLOT;
-                for (int h = 0; h < nb; ++h)
-                    if (rows[h]) {
-                        if constexpr (F8) {
-                            // e4m3 rows are 128 bytes: one 2-D box per block, blocks 8 KB apart
-                            tma_load_2d_elect(slot + h * 8192u, rows[h] == 64 ? &tm_k : &tm_k_rem, 0, first[h],
-                                              &x.k_full[s]);
-                        } else {
-                            load_block<D, IL>(slot + h * (IL ? L::BLOCK_IL : 64u * 128u), 128u * 128u, rows[h],
-                                              first[h], &tm_k, &tm_k_rem, &x.k_full[s]);
-                        }
+            constexpr int KB = 2 * KSLOTS;  // block slots
+            for (int e = 0; e < cnt; ++e) {
+                int first = 0;
+                const int rows = block_rows(a, list_entry(x.lst, lst, e), bh, &first);
+                if (rows == 0 && lane == 0) record_error(a.err, DEVERR_LIST | 2);
+                const int bi = e % KB;
+                if (!mbar_wait(&x.k_empty[bi], ((e / KB) & 1) ^ 1, abort_flag, a.err, 0x10)) break;
+                if (rows) mbar_arrive_expect_tx_elect(&x.k_full[bi], static_cast<uint32_t>(rows * 128 * L::NPQ));
+                else mbar_arrive_elect(&x.k_full[bi]);
+                uint8_t* slot = smem + L::OFF_K + ((e >> 1) % KSLOTS) * L::K_SLOT;
+                const int h = e & 1;
+                if (rows) {
+                    if constexpr (F8) {
+                        tma_load_2d_elect(slot + h * 8192u, rows == 64 ? &tm_k : &tm_k_rem, 0, first, &x.k_full[bi]);
+                    } else {
+                        load_block<D, IL>(slot + h * (IL ? L::BLOCK_IL : 64u * 128u), 128u * 128u, rows, first, &tm_k,
+                                          &tm_k_rem, &x.k_full[bi]);
                     }
-                armed = t + 1;
+                }
+                armed = e + 1;
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA exits.
                 mbar_drain(&x.q_full, 0, 10000000ull);
-                for (int t = max(0, armed - KSLOTS); t < armed; ++t)
-                    mbar_drain(&x.k_full[t % KSLOTS], (t / KSLOTS) & 1, 10000000ull);
+                for (int e = max(0, armed - KB); e < armed; ++e)
+                    mbar_drain(&x.k_full[e % KB], (e / KB) & 1, 10000000ull);
             }
         }
     } else if (warp == W_VPROD) {
@@ -371,7 +369,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // warp W_PV the PV MMAs; the waits below are normally already satisfied, which keeps
         // each issuing warp's code path short.
         {
-            constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(64, 128) : idesc_bf16_f32(64, 128, false, false);
+            constexpr uint32_t IDESC_S64 = F8 ? idesc_e4m3_f32(64, 64) : idesc_bf16_f32(64, 64, false, false);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64, true, false);
             // A descriptor's start field is the byte address >> 4, so an operand at a byte
             // offset o from a base is the base descriptor + (o >> 4).
@@ -389,27 +387,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (!mbar_wait(&x.s_free[bsel], ((st / SBUFS) - 1) & 1, abort_flag, a.err, 0x21)) return false;
                     tc_fence_after();  // the softmax's TMEM reads of this buffer come first
                 }
-                for (int h = 0; h < 2; ++h) {
-                    const int t = 2 * st + h;
-                    if (t >= n_tiles) break;
-                    const int ks = t % KSLOTS;
-                    if (!mbar_wait(&x.k_full[ks], (t / KSLOTS) & 1, abort_flag, a.err, 0x22)) return false;
-                    const uint32_t d_addr = tmem + 128u * static_cast<uint32_t>(bsel) + (h ? (16u << 16) : 0u);
-                    const uint64_t kb = dK + ((static_cast<uint32_t>(ks) * L::K_SLOT) >> 4);
+                for (int e = 4 * st; e < 4 * st + 4 && e < cnt; ++e) {
+                    constexpr int KB = 2 * KSLOTS;
+                    const int h = (e >> 1) & 1, b = e & 1;  // tile of the step, block of the tile
+                    const int bi = e % KB;
+                    if (!mbar_wait(&x.k_full[bi], (e / KB) & 1, abort_flag, a.err, 0x22)) return false;
+                    const uint32_t d_addr = tmem + 128u * static_cast<uint32_t>(bsel) + (h ? (16u << 16) : 0u) + 64u * b;
+                    const uint32_t boff = F8 ? 8192u : (IL ? L::BLOCK_IL : 64u * 128u);
+                    const uint64_t kb = dK + ((static_cast<uint32_t>((e >> 1) % KSLOTS) * L::K_SLOT + b * boff) >> 4);
                     if constexpr (F8) {
-                        // e4m3: K = 32 per MMA, one 128-byte row per operand row
 #pragma unroll
                         for (int kk = 0; kk < D / 32; ++kk)
-                            umma_f8_elect(d_addr, dQ + ((kk * 32) >> 4), kb + ((kk * 32) >> 4), IDESC_S, kk > 0 ? 1u : 0u);
+                            umma_f8_elect(d_addr, dQ + ((kk * 32) >> 4), kb + ((kk * 32) >> 4), IDESC_S64, kk > 0 ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oq = ((kk >> 2) * L::PANEL_Q + (kk & 3) * 32) >> 4;
                             const uint32_t ok_ = ((kk >> 2) * L::K_PANEL + (kk & 3) * 32) >> 4;
-                            umma_bf16_elect(d_addr, dQ + oq, kb + ok_, IDESC_S, kk > 0 ? 1u : 0u);
+                            umma_bf16_elect(d_addr, dQ + oq, kb + ok_, IDESC_S64, kk > 0 ? 1u : 0u);
                         }
                     }
-                    umma_commit_elect(&x.k_empty[ks]);
+                    umma_commit_elect(&x.k_empty[bi]);
                     issued_any = true;
                 }
                 umma_commit_elect(&x.s_full[bsel]);

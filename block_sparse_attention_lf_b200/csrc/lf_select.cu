@@ -18,8 +18,10 @@
 //   * frames: top-k by k rounds of warp arg-max over the keys;
 //   * blocks: top-k by rank counting (rank = number of larger keys), then a
 //     ballot/popc compaction writes the kept block ids in ascending order.
-// The one-dimensional variant (global block top-k, no frame level) takes one
-// CTA per scored row instead; see select_blocks_1d_kernel.
+// Both levels run in one launch (select_fused_kernel, one CTA per scored row). The
+// one-dimensional variant (global block top-k, no frame level) scores tiles of rows
+// of one head through a bulk-copy ring (select_1d_tile_kernel), or one row per CTA for
+// heads of more than 2,048 blocks (select_blocks_1d_kernel).
 #include "lf_device.cuh"
 #include "lf_internal.h"
 #include "lf_score.cuh"
@@ -30,6 +32,10 @@ namespace {
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int SEL_FUSED_MAX_WARPS = 16;
+// warps per fused-selection CTA: few warps keep every row's CTA resident at once (900 rows
+// at 10 CTAs per SM); 3 warps: 19.5 us at layer480p and 25.6 us at long-video against
+// 23.6 / 49.2 us with one warp per selected frame (9), lists unchanged
+constexpr int SEL_FUSED_WARPS = 3;
 
 // T_r of scored row `row` (one warp): frame scores of the memory frames, top-k_f by
 // warp arg-max rounds, forced frames added; written ascending to out (global) and, when
@@ -634,7 +640,7 @@ template <int D, int KPLF, int KPLB>
 cudaError_t launch_fused_k(const SelectFramesArgs& fa, const SelectBlocksArgs& ba, cudaStream_t s)
 {
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(fa.BH) * fa.Rq);
-    const int warps = ba.n_sel < SEL_FUSED_MAX_WARPS ? ba.n_sel : SEL_FUSED_MAX_WARPS;
+    const int warps = ba.n_sel < SEL_FUSED_WARPS ? ba.n_sel : SEL_FUSED_WARPS;
     select_fused_kernel<D, KPLF, KPLB><<<grid, 32 * warps, static_cast<size_t>(fa.n_sel) * sizeof(int), s>>>(fa, ba);
     return cudaGetLastError();
 }
