@@ -161,6 +161,28 @@ __device__ __forceinline__ void tma_load_4d_elect(void* smem_dst, const CUtensor
 // 1-D bulk copy (TMA, no tensor map) of `bytes` from global memory to shared memory,
 // completing on `bar`; one elected lane of a converged warp issues it. Both addresses
 // 16-byte aligned, bytes a multiple of 16.
+// An L2 policy that makes the lines it touches the first to be evicted: for data a kernel
+// streams once, so it replaces its own lines instead of other (possibly dirty) ones.
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// bulk_load_elect with an L2 cache policy for the source lines.
+__device__ __forceinline__ void bulk_load_elect_hint(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                     uint64_t policy)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n\t}" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_load_elect(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar)
 {
     asm volatile(
