@@ -209,30 +209,30 @@ __global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(
 // ---- one-dimensional selection, tiled, through a bulk-copy ring ----------------------
 // One CTA per tile of TR_ROWS scored rows (query blocks) of one head. A producer warp
 // streams the head's pooled keys in groups of 32 candidates (16 KB at head_dim 128) into a
-// TR_SLOTS-slot shared-memory ring with 1-D bulk copies, so each pooled key crosses
-// L2 -> SM once per tile instead of once per row. Consumer warp w scores rows 2(w % 4) and
-// 2(w % 4) + 1 against the groups g with g % 2 == w / 4: each candidate slice read from
-// shared memory feeds two inner products. Groups are laid out as in the one-row kernel
-// (32 consecutive blocks from the head's first), so every score, and with it every list,
-// is bit-identical to its. Slot s only ever holds groups of parity s % 2 and is consumed by
-// the same four warps, in order. (The two-level selection tiled the same way, all of a
-// head's blocks scored per tile, ran at 34.8 us against 23.6 us for select_fused_kernel,
-// which scores only the selected frames' blocks; it was not kept.)
+// shared-memory ring with 1-D bulk copies, so each pooled key crosses L2 -> SM once per tile
+// instead of once per row. CONS consumer warps form CONS / 4 classes of four; warp w scores
+// rows 2(w % 4) and 2(w % 4) + 1 against the groups g with g % (CONS / 4) == w / 4: each
+// candidate slice read from shared memory feeds two inner products, and the classes work on
+// different groups at once (the scoring is latency-bound: 16 warps score a tile about twice
+// as fast as 8). The ring has CONS / 2 slots, two per class; slot s only ever holds groups of
+// class s % (CONS / 4) and is consumed by the same four warps, in order. Groups are laid out
+// as in the one-row kernel (32 consecutive blocks from the head's first), so every score, and
+// with it every list, is bit-identical to its. (The two-level selection tiled the same way,
+// all of a head's blocks scored per tile, ran at 34.8 us against 23.6 us for
+// select_fused_kernel, which scores only the selected frames' blocks; it was not kept.)
 constexpr int TR_ROWS = 8;
-constexpr int TR_CONSUMERS = 8;
-constexpr int TR_CT = 32 * TR_CONSUMERS;  // consumer threads
-constexpr int TR_THREADS = TR_CT + 32;    // + the producer warp
-constexpr int TR_SLOTS = 4;               // even: slot s holds groups of parity s % 2
-constexpr int TR_1D_MAX_NKV = 2048;       // scores of a row in registers (64 per lane); beyond: the one-row kernel
+constexpr int TR_1D_MAX_NKV = 2048;  // scores of a row in registers (64 per lane); beyond: the one-row kernel
 
-template <int D>
+template <int D, int CONS>
 constexpr size_t tr_ring_bytes()
 {
-    return static_cast<size_t>(TR_SLOTS) * 32u * D * sizeof(float);
+    return static_cast<size_t>(CONS / 2) * 32u * D * sizeof(float);
 }
 
+template <int CONS>
 struct TileRing {
-    uint64_t full[TR_SLOTS], empty[TR_SLOTS];
+    static constexpr int SLOTS = CONS / 2;
+    uint64_t full[SLOTS], empty[SLOTS];
     int abort;
 };
 
@@ -271,20 +271,23 @@ __device__ __forceinline__ void score_group2(const float (&q0)[D / 32], const fl
     s1 = p1[0];
 }
 
-__device__ __forceinline__ void tile_ring_init(TileRing& r)
+template <int CONS>
+__device__ __forceinline__ void tile_ring_init(TileRing<CONS>& r)
 {
-    for (int s = 0; s < TR_SLOTS; ++s) {
+    for (int s = 0; s < TileRing<CONS>::SLOTS; ++s) {
         mbar_init(&r.full[s], 1);
-        mbar_init(&r.empty[s], TR_CONSUMERS / 2);  // the four warps of the slot's parity
+        mbar_init(&r.empty[s], 4);  // the four warps of the slot's class
     }
     r.abort = 0;
     fence_mbar_init();
 }
 
 // Producer warp: every group of the head, in order.
-template <int D>
-__device__ __forceinline__ void tile_produce(TileRing& r, const TileGroups& tg, const float* kblk, float* ring, int* err)
+template <int D, int CONS>
+__device__ __forceinline__ void tile_produce(TileRing<CONS>& r, const TileGroups& tg, const float* kblk, float* ring,
+                                             int* err)
 {
+    constexpr int TR_SLOTS = TileRing<CONS>::SLOTS;
     volatile int* abort_flag = &r.abort;
     int g = 0;
     for (; g < tg.n_groups; ++g) {
@@ -302,12 +305,13 @@ __device__ __forceinline__ void tile_produce(TileRing& r, const TileGroups& tg, 
 // Consumer warps: the tile's scores into sc[TR_ROWS][n]; rows past rows_valid score with a
 // zero query and are never read. Returns false when the CTA gave up; the answer is the same
 // in every consumer thread, and the call is the barrier after which sc is complete.
-template <int D>
-__device__ __forceinline__ bool tile_score(TileRing& r, const TileGroups& tg, const float* q_pool, long long row0,
+template <int D, int CONS>
+__device__ __forceinline__ bool tile_score(TileRing<CONS>& r, const TileGroups& tg, const float* q_pool, long long row0,
                                            int rows_valid, int n, const float* ring, float* sc, int* err, int warp,
                                            int lane)
 {
     constexpr int EPL = D / 32;
+    constexpr int TR_SLOTS = TileRing<CONS>::SLOTS;
     volatile int* abort_flag = &r.abort;
     const int ra = 2 * (warp & 3), rb = ra + 1, par = warp >> 2;
     float q0[EPL], q1[EPL];
@@ -318,7 +322,7 @@ __device__ __forceinline__ bool tile_score(TileRing& r, const TileGroups& tg, co
     }
     if (ra < rows_valid) load_lane<EPL>(q0, q_pool + (row0 + ra) * D + lane * EPL);
     if (rb < rows_valid) load_lane<EPL>(q1, q_pool + (row0 + rb) * D + lane * EPL);
-    for (int g = par; g < tg.n_groups; g += 2) {
+    for (int g = par; g < tg.n_groups; g += CONS / 4) {
         const int s = g % TR_SLOTS;
         if (!mbar_wait(&r.full[s], static_cast<uint32_t>((g / TR_SLOTS) & 1), abort_flag, err, 0x53)) break;
         const int base = tg.base(g), cnt = tg.count(g);
@@ -331,21 +335,21 @@ __device__ __forceinline__ bool tile_score(TileRing& r, const TileGroups& tg, co
         __syncwarp();
         if (lane == 0) mbar_arrive(&r.empty[s]);
     }
-    return !named_bar_or(1, TR_CT, *abort_flag != 0);
+    return !named_bar_or(1, 32 * CONS, *abort_flag != 0);
 }
 
 // One-dimensional selection over the tile's scores: each warp its row, the row's scores in
 // registers (VPL per lane, candidate 32 i + lane in slot i); the threshold score T of the
 // kept count is built bit by bit (32 rounds of per-lane counts and one warp reduction), then
 // every candidate above T and the lowest-indexed ones equal to T are written in index order.
-template <int D, int VPL>
-__global__ void __launch_bounds__(TR_THREADS) select_1d_tile_kernel(const SelectBlocks1dArgs a)
+template <int D, int VPL, int CONS>
+__global__ void __launch_bounds__(32 * CONS + 32) select_1d_tile_kernel(const SelectBlocks1dArgs a)
 {
     extern __shared__ __align__(128) uint8_t tr_smem[];
-    __shared__ TileRing rc;
+    __shared__ TileRing<CONS> rc;
     const int n = a.Nkv;
     float* ring = reinterpret_cast<float*>(tr_smem);
-    float* sc = reinterpret_cast<float*>(tr_smem + tr_ring_bytes<D>());  // [TR_ROWS][n]
+    float* sc = reinterpret_cast<float*>(tr_smem + tr_ring_bytes<D, CONS>());  // [TR_ROWS][n]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int tiles = (a.Rq + TR_ROWS - 1) / TR_ROWS;
     const int bh = static_cast<int>(blockIdx.x / tiles);
@@ -364,11 +368,11 @@ __global__ void __launch_bounds__(TR_THREADS) select_1d_tile_kernel(const Select
     const TileGroups tg(n);
     if (threadIdx.x == 0) tile_ring_init(rc);
     __syncthreads();
-    if (warp == TR_CONSUMERS) {
-        tile_produce<D>(rc, tg, a.k_pool + static_cast<long long>(bh) * n * D, ring, a.err);
+    if (warp == CONS) {
+        tile_produce<D, CONS>(rc, tg, a.k_pool + static_cast<long long>(bh) * n * D, ring, a.err);
         return;
     }
-    if (!tile_score<D>(rc, tg, a.q_pool, row0, rows_valid, n, ring, sc, a.err, warp, lane)) return;
+    if (!tile_score<D, CONS>(rc, tg, a.q_pool, row0, rows_valid, n, ring, sc, a.err, warp, lane)) return;
     if (warp >= rows_valid) return;
     const long long row = row0 + warp;
     int* out = a.block_list + row * a.list_cap;
@@ -569,17 +573,32 @@ cudaError_t tile_smem_optin(Kernel k, int& configured_device, size_t bytes)
     return cudaSuccess;
 }
 
+template <int D, int VPL, int CONS>
+cudaError_t launch_1d_tile_c(const SelectBlocks1dArgs& a, long long grid, cudaStream_t s)
+{
+    static int configured_device = -1;
+    cudaError_t e = tile_smem_optin(select_1d_tile_kernel<D, VPL, CONS>, configured_device,
+                                    tr_ring_bytes<D, CONS>() + TR_ROWS * TR_1D_MAX_NKV * sizeof(float));
+    if (e != cudaSuccess) return e;
+    select_1d_tile_kernel<D, VPL, CONS><<<static_cast<unsigned>(grid), 32 * CONS + 32,
+                                          tr_ring_bytes<D, CONS>() + static_cast<size_t>(TR_ROWS) * a.Nkv * sizeof(float),
+                                          s>>>(a);
+    return cudaGetLastError();
+}
+
+// 16 consumer warps (a 128 KB ring at head_dim 128, one CTA per SM) when the tiles fit in one
+// wave; otherwise 8 (a 64 KB ring, two CTAs per SM).
 template <int D, int VPL>
 cudaError_t launch_1d_tile(const SelectBlocks1dArgs& a, cudaStream_t s)
 {
-    static int configured_device = -1;
-    cudaError_t e = tile_smem_optin(select_1d_tile_kernel<D, VPL>, configured_device,
-                                    tr_ring_bytes<D>() + TR_ROWS * TR_1D_MAX_NKV * sizeof(float));
+    const long long grid = static_cast<long long>(a.BH) * ((a.Rq + TR_ROWS - 1) / TR_ROWS);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const long long tiles = (a.Rq + TR_ROWS - 1) / TR_ROWS;
-    select_1d_tile_kernel<D, VPL><<<static_cast<unsigned>(static_cast<long long>(a.BH) * tiles), TR_THREADS,
-                                    tr_ring_bytes<D>() + static_cast<size_t>(TR_ROWS) * a.Nkv * sizeof(float), s>>>(a);
-    return cudaGetLastError();
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (grid <= sms) return launch_1d_tile_c<D, VPL, 16>(a, grid, s);
+    return launch_1d_tile_c<D, VPL, 8>(a, grid, s);
 }
 
 template <int D>

@@ -76,6 +76,8 @@ CASES = [
     # many candidates per row (1,600 and 6,480 KV blocks of 8 per frame)
     ("1600_candidates", 1, 1, 64, 512, (1, 195, 1, 3), 2, 40),
     ("6480_candidates", 1, 1, 64, 512, (1, 805, 1, 3), 2, 50),
+    # 32 heads x 5 tiles of 8 query blocks: more tiles than SMs (the 8-warp ring)
+    ("160_tiles", 4, 8, 64, 256, (1, 3, 1, 10), 2, 9),
 ]
 
 
