@@ -51,7 +51,8 @@ def _args():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the per-config report (all five workloads, rollout per chunk)")
     p.add_argument("--config-steps", type=int, default=30)
-    p.add_argument("--only-report", choices=["layer480p_1d", "layer480p_fp8", "longvideo480p_ivf"], default=None,
+    p.add_argument("--only-report", choices=["layer480p_1d", "layer480p_fp8", "longvideo480p_ivf", "cached_pooled_keys"],
+                   default=None,
                    help="run only this extra report after the main line (skips the other configs); "
                         "used to profile one of its kernels")
     p.add_argument("--strong", action="store_true",
@@ -718,7 +719,10 @@ def run_ours(a):
         "wall_s_timed_region": wall,
     }
     extra = (("layer480p_1d", one_dim_report), ("layer480p_fp8", fp8_report), ("longvideo480p_ivf", ivf_report))
-    if rank == 0 and a.only_report:
+    if rank == 0 and a.only_report == "cached_pooled_keys":
+        mc = measure_call(L, shape, w.chunk_index, w.topk_frames, kb, q, k, v, a.config_steps, 3, flush, cached=True)
+        line["cached_pooled_keys"] = _summary(mc, peaks)
+    elif rank == 0 and a.only_report:
         line["configs"] = {}
         for key, fn in extra:
             if key == a.only_report:
