@@ -229,6 +229,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // the merge kernel of a split call may be scheduled once every CTA has started
     // (it waits for this grid's completion before reading anything)
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // launched as a programmatic dependent of the selection: its lists (and any earlier
+    // kernel's q, k, v) are complete and visible once this returns
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int row = blockIdx.x;
     int slot = -1;  // partial-result slot of a CTA that computes one piece of a list
     if (a.pieces > 0 && row >= a.n_whole) {
@@ -777,9 +780,21 @@ cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t s)
     }
     const int tail = a.pieces > 0 ? a.n_rows - a.n_whole : 0;
     const long long grid = a.n_units;
-    attn_kernel<D, IL, F8><<<static_cast<unsigned>(grid), ATTN_THREADS, smem, s>>>(m.q, m.q_rem, m.k, m.k_rem, m.v,
-                                                                             m.v_rem, a);
-    e = cudaGetLastError();
+    {
+        // a programmatic dependent launch: the grid may be scheduled while the previous kernel
+        // in the stream finishes, and waits for it (griddepcontrol.wait) before reading memory
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(ATTN_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, attn_kernel<D, IL, F8>, m.q, m.q_rem, m.k, m.k_rem, m.v, m.v_rem, a);
+    }
     if (e != cudaSuccess || tail == 0) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tail) * 8u);

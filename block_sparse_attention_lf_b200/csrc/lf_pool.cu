@@ -67,6 +67,8 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const PoolArgs a,
     uint64_t* empty = full + POOL_SLOTS;
     int* abort_word = reinterpret_cast<int*>(empty + POOL_SLOTS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the selection that follows may be scheduled now; it waits for this grid's completion
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int s = 0; s < POOL_SLOTS; ++s) {
             mbar_init(&full[s], 1);

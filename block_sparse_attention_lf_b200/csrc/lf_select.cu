@@ -197,6 +197,10 @@ __global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(
 {
     constexpr int EPL = D / 32;
     extern __shared__ int sel_s[];  // [n_sel]
+    // a programmatic dependent of the pooling: wait for its outputs, and let the attention
+    // that follows be scheduled early (it waits for this grid the same way)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
     const long long row = blockIdx.x;
     float qv[EPL];
@@ -660,8 +664,17 @@ cudaError_t launch_fused_k(const SelectFramesArgs& fa, const SelectBlocksArgs& b
 {
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(fa.BH) * fa.Rq);
     const int warps = ba.n_sel < SEL_FUSED_WARPS ? ba.n_sel : SEL_FUSED_WARPS;
-    select_fused_kernel<D, KPLF, KPLB><<<grid, 32 * warps, static_cast<size_t>(fa.n_sel) * sizeof(int), s>>>(fa, ba);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * warps);
+    cfg.dynamicSmemBytes = static_cast<size_t>(fa.n_sel) * sizeof(int);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see select_fused_kernel
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_fused_kernel<D, KPLF, KPLB>, fa, ba);
 }
 
 template <int D, int KPLF>
