@@ -284,3 +284,36 @@ def test_fused_selection_equals_two_kernels(name, chunk):
     assert torch.equal(b.frame_sel, fs2) and torch.equal(b.block_count, bc2)
     cnt = int(bc2.max())
     assert torch.equal(b.block_list[..., :cnt], bl2[..., :cnt])
+
+
+def test_dependent_launches_see_their_producers():
+    """The selection and the attention are launched as programmatic dependents of the kernel
+    before them and wait for it before reading. Back-to-back calls with no host
+    synchronisation, each preceded by a torch kernel that rewrites q, k and v, must give
+    every call the output of its own inputs: the output of each call equals the output of
+    the same inputs run alone (bit for bit, the same kernels)."""
+    import block_sparse_attention_lf_b200 as L
+    w = lf_synth.CONFIGS["layer480p"]
+    shape = L.shape_from_workload(w)
+    n_sel = L.lf_frames_selected(shape, w.chunk_index, w.topk_frames)
+    kb = w.topk_blocks or L.lf_blocks_for_sparsity(w.sparsity, shape.Nkv, n_sel, shape.bpf)
+    q0, k0, v0 = (t.cuda() for t in lf_synth.make_qkv(w))
+    call = L.HSACall(shape, w.chunk_index, w.topk_frames, kb)
+    scales = (1.0, -0.5, 2.0)
+    alone = []
+    for sc in scales:
+        call(q0 * sc, k0 * sc, v0 * sc)
+        torch.cuda.synchronize()
+        alone.append(call.buf.out.clone())
+    q, k, v = torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0)
+    chained = []
+    for sc in scales:
+        torch.mul(q0, sc, out=q)
+        torch.mul(k0, sc, out=k)
+        torch.mul(v0, sc, out=v)
+        call(q, k, v)
+        chained.append(call.buf.out.clone())  # a torch kernel after the attention's merge
+    torch.cuda.synchronize()
+    assert L.lf_get_device_error()[0] == 0
+    for a, c in zip(alone, chained):
+        assert torch.equal(a, c)
