@@ -381,6 +381,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
     asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrival at barrier `id` without waiting (a producer's release to the threads that sync on it).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads)
+{
+    asm volatile("barrier.cta.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // OR-reduction of a predicate over the `nthreads` threads of barrier `id`.
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred)
 {

@@ -33,9 +33,11 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int SEL_FUSED_MAX_WARPS = 16;
 // warps per fused-selection CTA: few warps keep every row's CTA resident at once (900 rows
-// at 10 CTAs per SM); 3 warps: 19.5 us at layer480p and 25.6 us at long-video against
-// 23.6 / 49.2 us with one warp per selected frame (9), lists unchanged
-constexpr int SEL_FUSED_WARPS = 3;
+// at 6-7 CTAs per SM). With the forced slots scored beside the frame level, 4 warps took
+// 18.4 / 20.5 / 29.6 us at layer480p / longvideo480p / patterns480p against 20.5 / 22.5 /
+// 32.8 us for 3 warps and 22.5 / 26.6 / 30.7 us for 5 (the frame level first, then all
+// slots, on 3 warps: 18.5 / 24.6 / 32.8 us); one warp per selected frame (9) was slower still.
+constexpr int SEL_FUSED_WARPS = 4;
 
 // T_r of scored row `row` (one warp): frame scores of the memory frames, top-k_f by
 // warp arg-max rounds, forced frames added; written ascending to out (global) and, when
@@ -186,28 +188,69 @@ __global__ void __launch_bounds__(SEL_THREADS) select_blocks_kernel(const Select
     blocks_of_frame<D, KPL>(a, row, s, tau, lane, qv);
 }
 
-// Both levels for one scored row per CTA, in one launch: warp 0 picks T_r (to frame_sel
-// and to shared memory), then warp w takes the blocks of selected frames w, w + W, ...
-// The arithmetic is the two kernels' above, so the result is bit-identical to
-// select_frames_kernel followed by select_blocks_kernel; the second launch and its
-// dependent gap are gone.
+// Both levels for one scored row per CTA, in one launch. The forced frames' slots of T_r
+// (sinks, recent and current frames) are known before the frame level, so while warp 0
+// picks T_r (to frame_sel and to shared memory) the other warps already take the block
+// top-k of those slots; the selected memory frames' slots follow once warp 0 has published
+// them (barrier 1: warp 0 arrives, every other warp syncs once). Slots are handed out in
+// that order from a shared counter. The arithmetic is the two kernels' above, so the result
+// is bit-identical to select_frames_kernel followed by select_blocks_kernel.
 template <int D, int KPLF, int KPLB>
 __global__ void __launch_bounds__(SEL_FUSED_MAX_WARPS * 32) select_fused_kernel(const SelectFramesArgs fa,
                                                                                 const SelectBlocksArgs ba)
 {
     constexpr int EPL = D / 32;
     extern __shared__ int sel_s[];  // [n_sel]
+    __shared__ int next_slot;
     // a programmatic dependent of the pooling: wait for its outputs, and let the attention
     // that follows be scheduled early (it waits for this grid the same way)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0) {
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        next_slot = 0;
+    }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
     const long long row = blockIdx.x;
     float qv[EPL];
     load_lane<EPL>(qv, fa.q_pool + row * D + lane * EPL);
-    if (warp == 0) frames_of_row<D, KPLF>(fa, row, lane, qv, fa.frame_sel + row * fa.n_sel, sel_s);
-    __syncthreads();
-    for (int s = warp; s < ba.n_sel; s += n_warps) blocks_of_frame<D, KPLB>(ba, row, s, sel_s[s], lane, qv);
+    // items [0, n_forced) are the forced slots in slot order, then the kf selected ones
+    int kf = 0;
+    if (fa.chunk_index != 1) {
+        const int n_mem = fa.NF - fa.n_sink - fa.n_recent - fa.n_cur;
+        kf = fa.topk < n_mem ? fa.topk : n_mem;
+    }
+    const int n_forced = ba.n_sel - kf;
+    const int tail0 = fa.NF - fa.n_recent - fa.n_cur;
+    const int bar_threads = 32 * n_warps;
+    __syncthreads();  // next_slot is initialised
+    bool synced = true;
+    if (warp == 0) {
+        frames_of_row<D, KPLF>(fa, row, lane, qv, fa.frame_sel + row * fa.n_sel, sel_s);
+        __syncwarp();
+        if (n_warps > 1) named_bar_arrive(1, bar_threads);
+    } else {
+        synced = false;
+    }
+    for (;;) {
+        int it = 0;
+        if (lane == 0) it = atomicAdd(&next_slot, 1);
+        it = __shfl_sync(0xffffffffu, it, 0);
+        if (it >= ba.n_sel) break;
+        int s, tau;
+        if (it < n_forced) {
+            s = it < fa.n_sink ? it : it + kf;
+            tau = (fa.chunk_index == 1 || s < fa.n_sink) ? s : tail0 + (s - fa.n_sink - kf);
+        } else {
+            if (!synced) {
+                named_bar_sync(1, bar_threads);
+                synced = true;
+            }
+            s = fa.n_sink + (it - n_forced);
+            tau = sel_s[s];
+        }
+        blocks_of_frame<D, KPLB>(ba, row, s, tau, lane, qv);
+    }
+    if (!synced) named_bar_sync(1, bar_threads);
 }
 
 // ---- one-dimensional selection, tiled, through a bulk-copy ring ----------------------
