@@ -58,6 +58,10 @@ SMALL = [
     ("no_sink_no_recent", 1, 2, 64, 256, (0, 5, 0, 2), 2, 2, 3, 1.0, 0),
     ("sharp_softmax_rescales", 1, 2, 128, 300, (1, 4, 1, 2), 2, 3, 3, 8.0, 0),
     ("long_lists_many_tiles", 1, 2, 128, 1560, (1, 7, 1, 1), 2, 7, 25, 1.0, 0),
+    # fewer selected frames than the fused selection's warps: one, two and three slots
+    ("single_frame_dense", 1, 2, 128, 100, (0, 0, 0, 1), 1, 1, 2, 1.0, 0),
+    ("two_slots", 1, 2, 128, 150, (0, 1, 0, 1), 2, 1, 2, 1.0, 0),
+    ("three_slots", 2, 2, 64, 90, (1, 1, 0, 1), 2, 1, 1, 1.0, 0),
 ]
 
 
@@ -251,7 +255,8 @@ LARGE_SELECTION = [
 
 
 @pytest.mark.parametrize("name,chunk", [("ragged_d128", 2), ("ragged_d64_odd_lists", 2), ("dense_first_chunk", 1),
-                                        ("no_memory_frames", 2), ("layer480p", 2), ("longvideo480p", 2),
+                                        ("no_memory_frames", 2), ("single_frame_dense", 1), ("two_slots", 2),
+                                        ("three_slots", 2), ("layer480p", 2), ("longvideo480p", 2),
                                         ("200_memory_frames", 2), ("805_memory_frames", 2)])
 def test_fused_selection_equals_two_kernels(name, chunk):
     """lf_select_mask (both levels in one launch) writes exactly what lf_select_frames followed by
