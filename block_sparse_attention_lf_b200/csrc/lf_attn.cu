@@ -76,9 +76,10 @@ namespace {
 constexpr int ATTN_THREADS = 384;
 constexpr int W_KPROD = 0, W_VPROD = 1, W_MMA = 2, W_PV = 3, W_SOFT0 = 4;
 // K ring (tiles of two blocks) and V ring (single blocks). e4m3 K tiles take half the
-// bytes of bf16 ones, which leaves room for a deeper V ring.
+// bytes of bf16 ones: the e4m3 kernel holds four K tiles (eight blocks, 64 KB) and four V
+// blocks, 2-4 % faster than two K tiles with six V blocks or three with five.
 template <bool F8> struct Rings { static constexpr int K = 2, V = 4; };
-template <> struct Rings<true> { static constexpr int K = 2, V = 6; };
+template <> struct Rings<true> { static constexpr int K = 4, V = 4; };
 constexpr int SBUFS = 3;    // S buffers in TMEM (one per step in flight)
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;  // p may reach 2^8 before the stabiliser moves
 constexpr uint32_t TMEM_COLS = 512;         // S buffer b: columns 128*b; O^T of warpgroup g: 384 + 64*g
